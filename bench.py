@@ -1,0 +1,380 @@
+"""Benchmark of one Muon optimizer step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload square4096] [--impl ours|reference]
+
+A step is one pass of the whole hot path over the workload: momentum + Nesterov
++ Frobenius norm, five Newton-Schulz iterations (Gram, polynomial and update
+GEMMs on the tensor cores), and the in-place weight update, through the C ABI.
+Default workload: one 4096 x 4096 bf16 gradient with a power-law spectrum,
+fp32 weights and momentum, weight decay 0.1.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronise, timed with CUDA events on the launching stream; the
+per-kernel times come from events the library records around each launch on
+that same stream.  Under torchrun every rank runs its own replica of the
+workload (the step does not shard a single matrix) and the time is the maximum
+over ranks.  Rank 0 prints one JSON line.
+
+`value` is whole-job throughput in nominal Newton-Schulz TFLOP/s: 5 (4 m^2 n +
+2 m^3) FLOPs per matrix per step, times ranks, divided by the step time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as wl  # noqa: E402
+
+METRIC = "Muon step ms & NS5 TFLOP/s (frac of bf16 peak); momentum/apply HBM GB/s"
+UNIT = "TFLOP/s"
+L2_BYTES = 126 * 2 ** 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world: int, backend: str):
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1 and not dist.is_initialized():
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Maximum of a per-rank float over all ranks (identity when world == 1)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv",
+                                          "-lms", "200"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path).read().splitlines()[1:]:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1].split()[0]))
+                smax.append(float(parts[2].split()[0]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- workload accounting
+
+def elementwise_bytes(w: wl.Workload):
+    """Algorithmic HBM bytes of the two memory-bound kernels of one step.
+
+    momentum+norm: read G (2 or 4 B) and B (4 B), write B (4 B), the fp32 iterate
+    (4 B) and its bf16 operand copy (2 B) = 16 B/elem for bf16 gradients.
+    apply: read W (4 B) and the fp32 result O (4 B), write W (4 B) = 12 B/elem."""
+    g = 2 if w.grad_dtype == wl.BF16 else 4
+    return w.elements * (g + 4 + 4 + 4 + 2), w.elements * 12
+
+
+def update_gemm_flops(w: wl.Workload):
+    """FLOPs of one launch of the update GEMM X' = P X (+ aX): 2 m^2 n per matrix."""
+    tot = 0.0
+    for s in w.matrices:
+        m, n = min(s.rows, s.cols), max(s.rows, s.cols)
+        tot += 2.0 * m * m * n
+    return tot
+
+
+def host_tensors(w: wl.Workload, device):
+    import torch
+    W = [torch.from_numpy(x) for x in wl.weights(w)]
+    G = []
+    for g in wl.grads(w, 0):
+        t = torch.from_numpy(np.ascontiguousarray(g).view(np.int16)).view(torch.bfloat16) if w.grad_dtype == wl.BF16 \
+            else torch.from_numpy(g)
+        G.append(t)
+    return W, G
+
+
+def groups_of(w, W, G, B):
+    import muon_newton_schulz_04_b200 as mb
+    return [mb.Group(W=[W[k] for k in idx], G=[G[k] for k in idx], B=[B[k] for k in idx]) for (_, _, idx) in w.groups()]
+
+
+# ----------------------------------------------------------------------------- CPU oracle baseline
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(w: wl.Workload, ns_iters: int):
+    """Time the oracle on one matrix of the workload: momentum, Nesterov direction,
+    normalisation, `ns_iters` Newton-Schulz iterations and the update.  Returns
+    (seconds, nominal NS FLOPs done)."""
+    import oracle
+    k = max(range(w.count), key=lambda i: w.matrices[i].rows * w.matrices[i].cols)
+    spec = w.matrices[k]
+    W = wl.weight(w, k).astype(np.float64)
+    G = wl.widen(wl.grad(w, 0, k), w.grad_dtype)
+    B = np.zeros_like(W)
+    m, n = min(spec.rows, spec.cols), max(spec.rows, spec.cols)
+    t0 = time.perf_counter()
+    oracle.muon_step(W, G, B, lr=w.lr, momentum=w.momentum, nesterov=w.nesterov, weight_decay=w.weight_decay,
+                     ns_steps=ns_iters, eps=w.eps)
+    dt = time.perf_counter() - t0
+    return dt, ns_iters * (4.0 * m * m * n + 2.0 * m ** 3), f"matrix {k} ({spec.rows}x{spec.cols}), {ns_iters} NS iteration(s)"
+
+
+def cpu_baseline(w: wl.Workload):
+    dt, flops, what = oracle_sample(w, 1)
+    iters = 1
+    if dt < 4.0:               # grow to a ~10-30 s sample
+        iters = int(min(w.ns_steps, max(1, math.floor(12.0 / max(dt, 1e-3)))))
+        if iters > 1:
+            dt, flops, what = oracle_sample(w, iters)
+    return {"value": round(flops / dt / 1e12, 6), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"fp64 numpy oracle, one Muon step of {what} of the {w.key} workload; {dt:.1f} s"}
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args, w):
+    world, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    times, flops_done, what = [], 0.0, ""
+    for i in range(args.warmup + args.steps):
+        dt, fl, what = oracle_sample(w, 1)
+        if i >= args.warmup:
+            times.append(dt)
+            flops_done += fl
+    total = sum(times)
+    v = flops_done / total / 1e12
+    line = {"metric": METRIC, "value": round(v, 6), "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * total / len(times), 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.key, "matrices": w.count, "sample": what},
+            "cpu_baseline": {"value": round(v, 6), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+                             "sample": f"each step: {what}"},
+            "e2e": {"value": round(v, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w):
+    import torch
+    import muon_newton_schulz_04_b200 as mb
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    peaks, peak_src = load_peaks()
+
+    cfg = mb.config(lr=w.lr, momentum=w.momentum, nesterov=int(w.nesterov), weight_decay=w.weight_decay,
+                    ns_steps=w.ns_steps, eps=w.eps, precision=mb.PREC_BF16)
+    opt = mb.Muon(cfg, device=local)
+    Wh, Gh = host_tensors(w, dev)
+    W = [x.to(dev) for x in Wh]
+    G = [x.to(dev) for x in Gh]
+    B = [torch.zeros_like(x) for x in W]
+    groups = groups_of(w, W, G, B)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        opt.step(groups)
+    opt.sync()
+
+    # --- device-resident timed region
+    opt.timing(True)
+    opt.timing_read()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    clocks.start()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        opt.step(groups)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    clk = clocks.stop()
+    ms_total = ev0.elapsed_time(ev1)
+    phases = opt.timing_read()
+    opt.timing(False)
+    ms_total = max_over_ranks(ms_total, world, dev)
+    ms_step = ms_total / args.steps
+
+    flops_nom = w.ns_flops_nominal()
+    value = flops_nom * world / (ms_step * 1e-3) / 1e12
+    launches = sum(n for (_, n) in phases.values())
+    gemm_ms = sum(phases[k][0] for k in ("gram", "poly", "update")) / args.steps
+    ns_tflops = flops_nom / (gemm_ms * 1e-3) / 1e12
+    b_mom, b_app = elementwise_bytes(w)
+    mom_ms = phases["momentum_norm"][0] / max(phases["momentum_norm"][1], 1)
+    app_ms = phases["apply"][0] / max(phases["apply"][1], 1)
+    upd_ms = phases["update"][0] / max(phases["update"][1], 1)
+    upd_tflops = update_gemm_flops(w) / (upd_ms * 1e-3) / 1e12
+
+    # --- end to end through the host-buffer entry point (pinned host memory)
+    Whp = [x.clone().pin_memory() for x in Wh]
+    Bhp = [torch.zeros_like(x).pin_memory() for x in Whp]
+    Ghp = [x.clone().pin_memory() for x in Gh]
+    hgroups = groups_of(w, Whp, Ghp, Bhp)
+    e2e_steps = max(1, min(args.steps, 10))
+    opt.step_host(hgroups)
+    opt.sync()
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(e2e_steps):
+        opt.step_host(hgroups)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev) / e2e_steps
+    gbytes = 2 if w.grad_dtype == wl.BF16 else 4
+    h2d = w.elements * (gbytes + 4 + 4)
+    d2h = w.elements * (4 + 4)
+
+    ws_bytes = w.elements * (4 + 4 + gbytes) + sum(
+        min(s.rows, s.cols) * (max(s.rows, s.cols) * (2 + 2 + 4) + 2 * 2 * min(s.rows, s.cols)) for s in w.matrices)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.key, "matrices": w.count, "elements": w.elements,
+                   "shapes": sorted({f"{s.rows}x{s.cols}" for s in w.matrices}),
+                   "ns_steps": w.ns_steps, "grad_dtype": w.grad_dtype, "weight_dtype": "fp32", "momentum_dtype": "fp32",
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": f"working set {ws_bytes / 2**20:.0f} MiB > 126 MiB L2 (no flush)",
+                   "flops_per_step_nominal": flops_nom, "flops_per_step_symmetric": w.ns_flops_symmetric()},
+        "ns5_tflops": round(ns_tflops, 2),
+        "ns5_frac_of_bf16_peak": round(ns_tflops / peaks["bf16_tflops"], 4),
+        "momentum_gbs": round(b_mom / (mom_ms * 1e-3) / 1e9, 1),
+        "momentum_frac_of_hbm": round(b_mom / (mom_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "apply_gbs": round(b_app / (app_ms * 1e-3) / 1e9, 1),
+        "apply_frac_of_hbm": round(b_app / (app_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "phase_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
+        "roofline": {"kernel": "ns_gemm_tc_kernel<UPDATE> (X' = P X + aX)", "bound": "tensor",
+                     "achieved": round(upd_tflops, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(upd_tflops / peaks["bf16_tflops"], 4), "traffic": None,
+                     "peak_source": f"{peak_src} bf16 dense (burst)",
+                     "flops_per_launch": update_gemm_flops(w), "avg_launch_ms": round(upd_ms, 5)},
+        "e2e": {"value": round(flops_nom * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 3),
+                "api": "muon_step_host (pinned host W, G, B)"},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    traffic = os.environ.get("MUON_UPDATE_TRAFFIC_BYTES")
+    if traffic:
+        line["roofline"]["traffic"] = float(traffic)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    opt.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="square4096", choices=sorted(wl.BY_KEY))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)          # at least 3 untimed warm-up steps
+    w = wl.get(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

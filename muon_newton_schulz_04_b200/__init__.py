@@ -1,0 +1,284 @@
+"""Python binding of the B200 Muon step library (include/muon.h).
+
+Argument marshalling only: torch tensors are turned into raw pointers, sizes
+and the current CUDA stream, and every entry point of the C ABI is called by
+the same name.  All arithmetic runs in the CUDA kernels of libmuon_b200.so;
+there is no fallback.  If the shared library is missing, the first call raises.
+
+    import torch, muon_newton_schulz_04_b200 as mb
+    opt = mb.Muon(mb.config(lr=0.02, weight_decay=0.1))
+    opt.step([mb.Group(W=[w1, w2], G=[g1, g2], B=[b1, b2])])   # same-shape matrices per group
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+from typing import List, Optional, Sequence
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmuon_b200.so")
+
+MUON_OK, MUON_ERR_INVALID, MUON_ERR_UNSUPPORTED, MUON_ERR_OOM, MUON_ERR_CUDA, MUON_ERR_DEVICE_TIMEOUT = range(6)
+MUON_BF16, MUON_FP32 = 0, 1
+PREC_BF16, PREC_FP32_DEBUG = 0, 1
+SCALE_NONE, SCALE_MATCH_RMS, SCALE_CUSTOM = 0, 1, 2
+NS_GRAM, NS_POLY, NS_UPDATE = 0, 1, 2
+
+
+class MuonConfig(ctypes.Structure):
+    _fields_ = [("lr", ctypes.c_float), ("momentum", ctypes.c_float), ("weight_decay", ctypes.c_float),
+                ("eps", ctypes.c_float), ("rms_target", ctypes.c_float), ("nesterov", ctypes.c_int),
+                ("ns_steps", ctypes.c_int), ("ns_a", ctypes.c_float), ("ns_b", ctypes.c_float),
+                ("ns_c", ctypes.c_float), ("scale_mode", ctypes.c_int), ("precision", ctypes.c_int)]
+
+
+class _Group(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("cols", ctypes.c_int), ("count", ctypes.c_int),
+                ("grad_dtype", ctypes.c_int), ("scale", ctypes.c_float),
+                ("W", ctypes.POINTER(ctypes.c_void_p)), ("G", ctypes.POINTER(ctypes.c_void_p)),
+                ("B", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class _OrthoGroup(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("cols", ctypes.c_int), ("count", ctypes.c_int),
+                ("in_dtype", ctypes.c_int), ("M", ctypes.POINTER(ctypes.c_void_p)),
+                ("O", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class _PhaseArgs(ctypes.Structure):
+    _fields_ = [("phase", ctypes.c_int), ("precision", ctypes.c_int), ("m", ctypes.c_int), ("n", ctypes.c_int),
+                ("count", ctypes.c_int), ("alpha", ctypes.c_float), ("beta", ctypes.c_float),
+                ("x_op", ctypes.c_void_p), ("a_in", ctypes.c_void_p), ("x_master", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("out_op", ctypes.c_void_p)]
+
+
+_LIB: Optional[ctypes.CDLL] = None
+
+# name -> (restype, argtypes)
+_SIGNATURES = {
+    "muon_config_default": (None, [ctypes.POINTER(MuonConfig)]),
+    "muon_validate_config": (ctypes.c_int, [ctypes.POINTER(MuonConfig)]),
+    "muon_validate_groups": (ctypes.c_int, [ctypes.POINTER(_Group), ctypes.c_int]),
+    "muon_create": (ctypes.c_int, [ctypes.POINTER(MuonConfig), ctypes.c_int, ctypes.POINTER(ctypes.c_void_p)]),
+    "muon_set_config": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(MuonConfig)]),
+    "muon_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_Group), ctypes.c_int, ctypes.c_void_p]),
+    "muon_step_host": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_Group), ctypes.c_int, ctypes.c_void_p]),
+    "muon_orthogonalize": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_OrthoGroup), ctypes.c_int, ctypes.c_void_p]),
+    "muon_ns_phase_run": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_PhaseArgs), ctypes.c_void_p]),
+    "muon_sync": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "muon_last_norms": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_float), ctypes.c_int,
+                                       ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]),
+    "muon_last_update": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
+    "muon_timing_enable": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int]),
+    "muon_timing_read": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int),
+                                        ctypes.c_int, ctypes.c_void_p]),
+    "muon_destroy": (ctypes.c_int, [ctypes.c_void_p]),
+    "muon_last_error": (ctypes.c_char_p, [ctypes.c_void_p]),
+    "muon_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "muon_plan_tile_m": (ctypes.c_int, []),
+    "muon_plan_tile_n": (ctypes.c_int, []),
+    "muon_plan_tiles": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.c_int,
+                                       ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded C library.  Raises if libmuon_b200.so has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m muon_newton_schulz_04_b200.build` "
+                               "(there is no CPU fallback)")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _LIB = L
+    return _LIB
+
+
+class MuonError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{lib().muon_status_string(status).decode()}: {msg}")
+        self.status = status
+
+
+def config(**kw) -> MuonConfig:
+    """Default configuration (lr 0.02, momentum 0.95 Nesterov, 5 steps, (3.4445, -4.775, 2.0315), eps 1e-7)
+    with the given fields replaced."""
+    c = MuonConfig()
+    lib().muon_config_default(ctypes.byref(c))
+    for k, v in kw.items():
+        if k not in dict(MuonConfig._fields_):
+            raise TypeError(f"unknown config field {k}")
+        setattr(c, k, int(v) if isinstance(getattr(c, k), int) else float(v))
+    return c
+
+
+@dataclasses.dataclass
+class Group:
+    """Same-shape matrices: W (fp32, updated), G (bf16 or fp32), B (fp32 momentum, updated)."""
+    W: Sequence
+    G: Sequence
+    B: Sequence
+    scale: float = 1.0
+
+
+def _ptrs(ts) -> "ctypes.Array":
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = t.data_ptr()
+    return arr
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return MUON_BF16
+    if t.dtype == torch.float32:
+        return MUON_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _check_tensors(ts, shape, on_cuda: bool):
+    for t in ts:
+        if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+            raise ValueError(f"expected contiguous tensors of shape {tuple(shape)}, got {tuple(t.shape)}")
+        if t.is_cuda != on_cuda:
+            raise ValueError("tensor on the wrong device kind")
+
+
+def _stream(stream) -> int:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+class Muon:
+    """A handle of the C library bound to one CUDA device."""
+
+    def __init__(self, cfg: Optional[MuonConfig] = None, device: int = 0):
+        self._h = ctypes.c_void_p()
+        self.cfg = cfg if cfg is not None else config()
+        st = lib().muon_create(ctypes.byref(self.cfg), int(device), ctypes.byref(self._h))
+        if st != MUON_OK:
+            raise MuonError(st, f"muon_create on device {device}")
+        self.device = device
+        self._keep = []
+
+    # ------------------------------------------------------------------ helpers
+    def _check(self, st: int, what: str):
+        if st != MUON_OK:
+            raise MuonError(st, f"{what}: {lib().muon_last_error(self._h).decode()}")
+
+    def _groups(self, groups: List[Group], on_cuda: bool):
+        arr = (_Group * len(groups))()
+        keep = []
+        for i, g in enumerate(groups):
+            rows, cols = g.W[0].shape
+            _check_tensors(g.W, (rows, cols), on_cuda)
+            _check_tensors(g.G, (rows, cols), on_cuda)
+            _check_tensors(g.B, (rows, cols), on_cuda)
+            if not (len(g.W) == len(g.G) == len(g.B)):
+                raise ValueError("W, G and B lists differ in length")
+            pw, pg, pb = _ptrs(g.W), _ptrs(g.G), _ptrs(g.B)
+            keep += [pw, pg, pb]
+            arr[i] = _Group(rows, cols, len(g.W), _dtype_code(g.G[0]), float(g.scale),
+                            ctypes.cast(pw, ctypes.POINTER(ctypes.c_void_p)),
+                            ctypes.cast(pg, ctypes.POINTER(ctypes.c_void_p)),
+                            ctypes.cast(pb, ctypes.POINTER(ctypes.c_void_p)))
+        return arr, keep
+
+    # ------------------------------------------------------------------ API
+    def set_config(self, cfg: MuonConfig):
+        self._check(lib().muon_set_config(self._h, ctypes.byref(cfg)), "muon_set_config")
+        self.cfg = cfg
+
+    def step(self, groups: List[Group], stream=None):
+        arr, keep = self._groups(groups, True)
+        self._check(lib().muon_step(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream))), "muon_step")
+
+    def step_host(self, groups: List[Group], stream=None):
+        arr, keep = self._groups(groups, False)
+        self._check(lib().muon_step_host(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream))), "muon_step_host")
+
+    def orthogonalize(self, groups, stream=None):
+        """groups: list of (M_list, O_list); O = NS(M / (||M||_F + eps)), fp32 outputs."""
+        arr = (_OrthoGroup * len(groups))()
+        keep = []
+        for i, (Ms, Os) in enumerate(groups):
+            rows, cols = Ms[0].shape
+            _check_tensors(Ms, (rows, cols), True)
+            _check_tensors(Os, (rows, cols), True)
+            pm, po = _ptrs(Ms), _ptrs(Os)
+            keep += [pm, po]
+            arr[i] = _OrthoGroup(rows, cols, len(Ms), _dtype_code(Ms[0]),
+                                 ctypes.cast(pm, ctypes.POINTER(ctypes.c_void_p)),
+                                 ctypes.cast(po, ctypes.POINTER(ctypes.c_void_p)))
+        self._check(lib().muon_orthogonalize(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream))),
+                    "muon_orthogonalize")
+
+    def ns_phase(self, phase: int, precision: int, m: int, n: int, count: int, alpha: float, beta: float,
+                 x_op=None, a_in=None, x_master=None, out=None, out_op=None, stream=None):
+        p = lambda t: None if t is None else t.data_ptr()
+        args = _PhaseArgs(phase, precision, m, n, count, alpha, beta, p(x_op), p(a_in), p(x_master), p(out), p(out_op))
+        self._check(lib().muon_ns_phase_run(self._h, ctypes.byref(args), ctypes.c_void_p(_stream(stream))),
+                    "muon_ns_phase_run")
+
+    def sync(self, stream=None):
+        self._check(lib().muon_sync(self._h, ctypes.c_void_p(_stream(stream))), "muon_sync")
+
+    def last_norms(self, stream=None) -> List[float]:
+        n = ctypes.c_int(0)
+        lib().muon_last_norms(self._h, None, 0, ctypes.byref(n), ctypes.c_void_p(_stream(stream)))
+        buf = (ctypes.c_float * max(n.value, 1))()
+        self._check(lib().muon_last_norms(self._h, buf, n.value, ctypes.byref(n), ctypes.c_void_p(_stream(stream))),
+                    "muon_last_norms")
+        return list(buf[: n.value])
+
+    def last_update(self, group: int, index: int, dst, stream=None):
+        self._check(lib().muon_last_update(self._h, group, index, ctypes.c_void_p(dst.data_ptr()),
+                                           ctypes.c_void_p(_stream(stream))), "muon_last_update")
+
+    TIMING_KINDS = ("momentum_norm", "norm_finalize", "gram", "poly", "update", "apply")
+
+    def timing(self, enable: bool = True):
+        self._check(lib().muon_timing_enable(self._h, int(enable)), "muon_timing_enable")
+
+    def timing_read(self, stream=None):
+        """{phase: (total ms, launches)} since the last read (synchronises the stream)."""
+        k = len(self.TIMING_KINDS)
+        ms = (ctypes.c_double * k)()
+        n = (ctypes.c_int * k)()
+        self._check(lib().muon_timing_read(self._h, ms, n, k, ctypes.c_void_p(_stream(stream))), "muon_timing_read")
+        return {name: (ms[i], n[i]) for i, name in enumerate(self.TIMING_KINDS)}
+
+    def close(self):
+        if self._h:
+            lib().muon_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def plan_tiles(shapes, phase: int):
+    """Tile list of a grouped GEMM launch: [(group, matrix, tile_row, tile_col)] (host only)."""
+    flat = (ctypes.c_int * (3 * len(shapes)))(*[int(v) for s in shapes for v in s])
+    n = ctypes.c_int(0)
+    lib().muon_plan_tiles(flat, len(shapes), phase, None, 0, ctypes.byref(n))
+    out = (ctypes.c_int * (4 * max(n.value, 1)))()
+    st = lib().muon_plan_tiles(flat, len(shapes), phase, out, n.value, ctypes.byref(n))
+    if st != MUON_OK:
+        raise MuonError(st, "muon_plan_tiles")
+    return [tuple(out[4 * i: 4 * i + 4]) for i in range(n.value)]
+
+
+def tile_shape():
+    return lib().muon_plan_tile_m(), lib().muon_plan_tile_n()

@@ -1,0 +1,273 @@
+// elementwise.cu -- the memory-bound phases of the Muon step.
+//
+//  momentum_norm   B <- mu*B + G                    ("Muon: An optimizer for hidden layers
+//                  U <- G + mu*B (Nesterov) or B     in neural networks", section 4, eq. 1
+//                                                    and its Nesterov remark)
+//                  X0 <- U, or U^T when rows > cols  (section 4: smaller-Gram orientation)
+//                  per-block sum of U^2 in fp64      (section 4: Frobenius normalisation)
+//  norm_finalize   ||U||_F and s = 1/(||U||_F + eps) per matrix, summed in a fixed order
+//  apply           W <- (1 - lr*wd) W - lr*s_shape*O (eq. 3 with decoupled decay and the
+//                  per-shape scale of the Moonlight result), O read back transposed
+//                  when the matrix was oriented; or O copied out (orthogonalisation only)
+//
+// One launch covers every matrix of the call: the block index is mapped to its
+// matrix by a binary search over the per-matrix block ranges.  Square or wide
+// matrices take a flat path (8 elements per thread per access, 16/32-byte
+// vectors); tall matrices go through a 64x64 shared-memory transpose so that
+// both the row-major reads and the transposed writes stay coalesced.
+#include "kernels.cuh"
+
+namespace muon {
+namespace {
+
+__device__ __forceinline__ int find_seg(const EwSeg* segs, int nseg, int blk, bool apply) {
+    int lo = 0, hi = nseg - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        const int b = apply ? segs[mid].apply_begin : segs[mid].blk_begin;
+        if (b <= blk) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__device__ __forceinline__ double block_sum(double v, double* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
+    if (l == 0) red[w] = v;
+    __syncthreads();
+    double r = 0.0;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < EW_THREADS / 32; ++i) r += red[i];
+    }
+    return r;
+}
+
+__device__ __forceinline__ float load_g(const void* g, size_t i, int bf16) {
+    return bf16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(g)[i])
+                : reinterpret_cast<const float*>(g)[i];
+}
+
+__device__ __forceinline__ float direction(float g, float* bptr, float mu, int nesterov) {
+    if (bptr == nullptr) return g;                     // orthogonalisation only: U = M
+    const float bn = fmaf(mu, *bptr, g);               // eq. 1
+    *bptr = bn;
+    return nesterov ? fmaf(mu, bn, g) : bn;
+}
+
+__global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* __restrict__ segs, int nseg,
+                                                                  double* __restrict__ partials, float mu,
+                                                                  int nesterov, int bf16_operand) {
+    __shared__ float tile[EW_TILE][EW_TILE + 1];
+    __shared__ double red[EW_THREADS / 32];
+    const int si = find_seg(segs, nseg, blockIdx.x, false);
+    const EwSeg sg = segs[si];
+    const int lb = blockIdx.x - sg.blk_begin;
+    double acc = 0.0;
+    __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(sg.xb0);
+
+    if (!sg.transposed) {
+        const size_t total = (size_t)sg.rows * sg.cols;
+        const size_t e0 = (size_t)lb * EW_FLAT_ELEMS;
+        const size_t e1 = min(total, e0 + EW_FLAT_ELEMS);
+        if (sg.vec && sg.b != nullptr) {
+            // rows are dense and 8-aligned: the oriented X has the same flat index
+            for (size_t e = e0 + (size_t)threadIdx.x * 8; e < e1; e += (size_t)EW_THREADS * 8) {
+                float g[8], b[8], u[8];
+                if (sg.g_bf16) {
+                    const uint4 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(sg.g) + e);
+                    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        g[2 * i] = __uint_as_float(w[i] << 16);
+                        g[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+                    }
+                } else {
+                    const float4 a0 = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(sg.g) + e);
+                    const float4 a1 = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(sg.g) + e + 4);
+                    g[0] = a0.x; g[1] = a0.y; g[2] = a0.z; g[3] = a0.w; g[4] = a1.x; g[5] = a1.y; g[6] = a1.z; g[7] = a1.w;
+                }
+                float4* bp = reinterpret_cast<float4*>(sg.b + e);
+                const float4 b0 = bp[0], b1 = bp[1];
+                b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w; b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    b[i] = fmaf(mu, b[i], g[i]);
+                    u[i] = nesterov ? fmaf(mu, b[i], g[i]) : b[i];
+                    acc += (double)u[i] * (double)u[i];
+                }
+                bp[0] = make_float4(b[0], b[1], b[2], b[3]);
+                bp[1] = make_float4(b[4], b[5], b[6], b[7]);
+                float4* xp = reinterpret_cast<float4*>(sg.xf0 + e);
+                xp[0] = make_float4(u[0], u[1], u[2], u[3]);
+                xp[1] = make_float4(u[4], u[5], u[6], u[7]);
+                if (bf16_operand) {
+                    uint4 w;
+                    __nv_bfloat162 h0 = __floats2bfloat162_rn(u[0], u[1]), h1 = __floats2bfloat162_rn(u[2], u[3]);
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(u[4], u[5]), h3 = __floats2bfloat162_rn(u[6], u[7]);
+                    w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
+                    w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
+                    *reinterpret_cast<uint4*>(xb + e) = w;
+                }
+            }
+        } else {
+            for (size_t e = e0 + threadIdx.x; e < e1; e += EW_THREADS) {
+                const size_t r = e / (size_t)sg.cols, c = e - r * (size_t)sg.cols;
+                const float u = direction(load_g(sg.g, e, sg.g_bf16), sg.b ? sg.b + e : nullptr, mu, nesterov);
+                acc += (double)u * (double)u;
+                const size_t xo = r * (size_t)sg.ldn + c;
+                sg.xf0[xo] = u;
+                if (bf16_operand) xb[xo] = __float2bfloat16_rn(u);
+            }
+        }
+    } else {
+        // tall matrix: X = U^T.  Tile of U rows [i0, i0+64) x cols [j0, j0+64).
+        const int tiles_c = (sg.cols + EW_TILE - 1) / EW_TILE;
+        const int i0 = (lb / tiles_c) * EW_TILE, j0 = (lb % tiles_c) * EW_TILE;
+        const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;     // 64 x 4
+#pragma unroll 4
+        for (int ii = ty; ii < EW_TILE; ii += 4) {
+            const int i = i0 + ii, j = j0 + tx;
+            float u = 0.f;
+            if (i < sg.rows && j < sg.cols) {
+                const size_t e = (size_t)i * sg.cols + j;
+                u = direction(load_g(sg.g, e, sg.g_bf16), sg.b ? sg.b + e : nullptr, mu, nesterov);
+                acc += (double)u * (double)u;
+            }
+            tile[ii][tx] = u;
+        }
+        __syncthreads();
+        // write X[j][i] = U[i][j]: consecutive threads take consecutive i
+#pragma unroll 4
+        for (int jj = ty; jj < EW_TILE; jj += 4) {
+            const int j = j0 + jj, i = i0 + tx;
+            if (j < sg.cols && i < sg.rows) {
+                const float u = tile[tx][jj];
+                const size_t xo = (size_t)j * sg.ldn + i;
+                sg.xf0[xo] = u;
+                if (bf16_operand) xb[xo] = __float2bfloat16_rn(u);
+            }
+        }
+    }
+    const double tot = block_sum(acc, red);
+    if (threadIdx.x == 0) partials[blockIdx.x] = tot;
+}
+
+// One warp per matrix: fixed-order sum of its block partials.
+__global__ void norm_finalize_kernel(const EwSeg* __restrict__ segs, int nseg, const double* __restrict__ partials,
+                                     float eps, float* __restrict__ norms, float* __restrict__ scale) {
+    const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (wid >= nseg) return;
+    const EwSeg& sg = segs[wid];
+    double s = 0.0;
+    for (int i = lane; i < sg.blk_count; i += 32) s += partials[sg.blk_begin + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_down_sync(0xffffffffu, s, o);
+    if (lane == 0) {
+        const double nrm = sqrt(s);
+        norms[sg.mat] = (float)nrm;
+        scale[sg.mat] = (float)(1.0 / (nrm + (double)eps));
+    }
+}
+
+// Apply (copy_out == 0) or copy-out (copy_out == 1) for one block of one matrix.
+__device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay, float lr, const float* o_scale,
+                                            int copy_out, float* dst) {
+    __shared__ float tile[EW_TILE][EW_TILE + 1];
+    const float os = o_scale ? o_scale[sg.mat] : 1.0f;
+    const float step = lr * sg.update_scale;
+    if (!sg.transposed) {
+        const size_t total = (size_t)sg.rows * sg.cols;
+        const size_t e0 = (size_t)lb * EW_FLAT_ELEMS;
+        const size_t e1 = min(total, e0 + EW_FLAT_ELEMS);
+        if (sg.vec) {
+            for (size_t e = e0 + (size_t)threadIdx.x * 8; e < e1; e += (size_t)EW_THREADS * 8) {
+                const float4* op = reinterpret_cast<const float4*>(sg.o_src + e);
+                float4 o0 = op[0], o1 = op[1];
+                float4* wp = reinterpret_cast<float4*>(dst + e);
+                if (copy_out) {
+                    o0.x *= os; o0.y *= os; o0.z *= os; o0.w *= os; o1.x *= os; o1.y *= os; o1.z *= os; o1.w *= os;
+                    wp[0] = o0; wp[1] = o1;
+                } else {
+                    float4 w0 = wp[0], w1 = wp[1];
+                    w0.x = fmaf(-step, o0.x * os, decay * w0.x); w0.y = fmaf(-step, o0.y * os, decay * w0.y);
+                    w0.z = fmaf(-step, o0.z * os, decay * w0.z); w0.w = fmaf(-step, o0.w * os, decay * w0.w);
+                    w1.x = fmaf(-step, o1.x * os, decay * w1.x); w1.y = fmaf(-step, o1.y * os, decay * w1.y);
+                    w1.z = fmaf(-step, o1.z * os, decay * w1.z); w1.w = fmaf(-step, o1.w * os, decay * w1.w);
+                    wp[0] = w0; wp[1] = w1;
+                }
+            }
+        } else {
+            for (size_t e = e0 + threadIdx.x; e < e1; e += EW_THREADS) {
+                const size_t r = e / (size_t)sg.cols, c = e - r * (size_t)sg.cols;
+                const float o = sg.o_src[r * (size_t)sg.ldn + c] * os;
+                dst[e] = copy_out ? o : fmaf(-step, o, decay * dst[e]);
+            }
+        }
+    } else {
+        // O = X^T: read X rows j (coalesced over i), write W rows i (coalesced over j)
+        const int tiles_c = (sg.cols + EW_TILE - 1) / EW_TILE;
+        const int i0 = (lb / tiles_c) * EW_TILE, j0 = (lb % tiles_c) * EW_TILE;
+        const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
+#pragma unroll 4
+        for (int jj = ty; jj < EW_TILE; jj += 4) {
+            const int j = j0 + jj, i = i0 + tx;
+            tile[jj][tx] = (j < sg.cols && i < sg.rows) ? sg.o_src[(size_t)j * sg.ldn + i] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int ii = ty; ii < EW_TILE; ii += 4) {
+            const int i = i0 + ii, j = j0 + tx;
+            if (i < sg.rows && j < sg.cols) {
+                const size_t e = (size_t)i * sg.cols + j;
+                const float o = tile[tx][ii] * os;
+                dst[e] = copy_out ? o : fmaf(-step, o, decay * dst[e]);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(EW_THREADS) apply_kernel(const EwSeg* __restrict__ segs, int nseg, float decay,
+                                                          float lr, const float* __restrict__ o_scale, int copy_out) {
+    const int si = find_seg(segs, nseg, blockIdx.x, true);
+    const EwSeg sg = segs[si];
+    apply_block(sg, blockIdx.x - sg.apply_begin, decay, lr, o_scale, copy_out, sg.w);
+}
+
+__global__ void __launch_bounds__(EW_THREADS) copy_out_one_kernel(const EwSeg sg, float* dst, const float* o_scale) {
+    apply_block(sg, blockIdx.x, 1.0f, 0.0f, o_scale, 1, dst);
+}
+
+}  // namespace
+
+cudaError_t launch_momentum_norm(const EwSeg* segs, int nseg, int nblocks, double* partials, float mu,
+                                 int nesterov, int bf16_operand, cudaStream_t s) {
+    if (nblocks <= 0) return cudaSuccess;
+    momentum_norm_kernel<<<nblocks, EW_THREADS, 0, s>>>(segs, nseg, partials, mu, nesterov, bf16_operand);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_norm_finalize(const EwSeg* segs, int nseg, const double* partials, float eps, float* norms,
+                                 float* scale, cudaStream_t s) {
+    if (nseg <= 0) return cudaSuccess;
+    const int threads = 256;
+    const int blocks = (nseg * 32 + threads - 1) / threads;
+    norm_finalize_kernel<<<blocks, threads, 0, s>>>(segs, nseg, partials, eps, norms, scale);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_apply(const EwSeg* segs, int nseg, int nblocks, float decay, float lr, const float* o_scale,
+                         int copy_out, cudaStream_t s) {
+    if (nblocks <= 0) return cudaSuccess;
+    apply_kernel<<<nblocks, EW_THREADS, 0, s>>>(segs, nseg, decay, lr, o_scale, copy_out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_copy_out_one(const EwSeg& seg, float* dst, const float* o_scale, cudaStream_t s) {
+    if (seg.apply_count <= 0) return cudaSuccess;
+    copy_out_one_kernel<<<seg.apply_count, EW_THREADS, 0, s>>>(seg, dst, o_scale);
+    return cudaGetLastError();
+}
+
+}  // namespace muon

@@ -1,0 +1,112 @@
+// kernels.cuh -- device-side descriptors and kernel launchers of the Muon step.
+//
+// Layout in HBM (library-owned workspace, per group of same-shape matrices):
+//   xb[2]  bf16 [count][m][ldn]   operand copies of the iterate X (ping-pong)
+//   xf[.]  fp32 [count][m][ldn]   the iterate itself (1 buffer on the bf16 path,
+//                                 2 ping-pong buffers on the fp32 debug path)
+//   a, p   bf16 [count][m][ldm]   Gram matrix A = XX^T and P = bA + cA^2
+//                                 (fp32 on the debug path)
+// with m = min(rows, cols), n = max(rows, cols), ldm / ldn rounded up to 8
+// elements so that every row starts on a 16-byte boundary (a TMA requirement).
+// The caller's W, G, B stay where the caller put them.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+namespace muon {
+
+// GEMM tile shape of the tensor-core kernels: 128 x 256 output elements per
+// tile, 64-element K blocks (one 128-byte swizzle atom of bf16).
+constexpr int TC_BM = 128;
+constexpr int TC_BN = 256;
+constexpr int TC_BK = 64;
+
+enum GemmMode { MODE_GRAM = 0, MODE_POLY = 1, MODE_UPDATE = 2 };
+
+// Elementwise work unit: one matrix.  Built on the host whenever the caller's
+// pointers or the plan change.
+struct EwSeg {
+    const void* g;        // gradient (step) or input M (orthogonalize): rows x cols
+    float* b;             // momentum buffer (nullptr: no momentum, U = G)
+    float* w;             // weight (apply) or output O (copy-out)
+    float* xf0;           // fp32 iterate written by the momentum kernel (m x ldn)
+    void* xb0;            // bf16 operand copy written by the momentum kernel (nullptr on fp32 path)
+    const float* o_src;   // final fp32 iterate read by the apply kernel (m x ldn)
+    int rows, cols;       // of W
+    int ldn;              // row stride of the oriented iterate
+    int transposed;       // rows > cols: X = U^T
+    int g_bf16;           // gradient dtype
+    int vec;              // flat 8-wide vector path allowed
+    int blk_begin;        // first block of this matrix in the momentum launch (= partial index)
+    int blk_count;
+    int apply_begin;      // first block in the apply launch
+    int apply_count;
+    int mat;              // global matrix index (norm / scale arrays)
+    float update_scale;   // per-shape scale s of the update
+};
+
+struct alignas(64) GemmMaps {
+    CUtensorMap xb_k[2];   // X operand, box {64, 128}: rows of X (K-major operand)
+    CUtensorMap xb_mn[2];  // X operand, box {64, 64}: X as an N-contiguous operand
+    CUtensorMap a;         // A, box {64, 128}
+    CUtensorMap p;         // P, box {64, 128}
+};
+
+struct GemmGroupInfo {
+    int m, n, ldm, ldn;
+    int count;
+    int mat_base;                 // global index of this group's matrix 0
+    __nv_bfloat16* xb[2];
+    const float* xf_in;           // UPDATE: fp32 X read for the beta term
+    float* xf_out;                // UPDATE: fp32 X' written
+    __nv_bfloat16* a;             // GRAM output / POLY input
+    __nv_bfloat16* p;             // POLY output / UPDATE input (via map)
+};
+
+struct GemmParams {
+    const int4* tiles;            // (group, matrix, tile_row, tile_col), cost-descending
+    int ntiles;
+    const GemmMaps* maps;
+    const GemmGroupInfo* groups;
+    int parity;                   // which xb holds the current iterate
+    float alpha, beta;            // GRAM: alpha; POLY: alpha = c, beta = b; UPDATE: alpha = 1, beta = a
+    const float* scale;           // per-matrix 1/(||U||+eps) on the first iteration, else nullptr
+    int write_op;                 // UPDATE: also write the bf16 operand copy of X'
+    int* err;                     // device error word (bounded waits)
+};
+
+size_t tc_gemm_smem_bytes();
+int tc_gemm_threads();
+cudaError_t tc_gemm_prepare();    // sets the dynamic shared-memory attribute once per device
+cudaError_t launch_tc_gemm(int mode, const GemmParams& p, int grid, cudaStream_t s);
+
+// fp32 FFMA debug GEMM: C = alpha_eff * A op(B) + beta_eff * Cin, batched over `count`.
+// op(B)[k][j] = B[j][k] when b_kmajor, else B[k][j].  With `scale`, alpha_eff =
+// alpha * s^scale_pow and beta_eff = beta * s^scale_pow where s = scale[mat_base + z].
+struct SimtGemmArgs {
+    const float* A; const float* B; float* C; const float* Cin;
+    int M, N, K, lda, ldb, ldc, ldcin;
+    long long sA, sB, sC, sCin;
+    int count, b_kmajor;
+    float alpha, beta;
+    const float* scale; int scale_pow; int mat_base;
+};
+cudaError_t launch_simt_gemm(const SimtGemmArgs& a, cudaStream_t s);
+
+// Elementwise kernels.
+cudaError_t launch_momentum_norm(const EwSeg* segs, int nseg, int nblocks, double* partials,
+                                 float mu, int nesterov, int bf16_operand, cudaStream_t s);
+cudaError_t launch_norm_finalize(const EwSeg* segs, int nseg, const double* partials, float eps,
+                                 float* norms, float* scale, cudaStream_t s);
+cudaError_t launch_apply(const EwSeg* segs, int nseg, int nblocks, float decay, float lr,
+                         const float* o_scale, int copy_out, cudaStream_t s);
+cudaError_t launch_copy_out_one(const EwSeg& seg, float* dst, const float* o_scale, cudaStream_t s);
+
+constexpr int EW_THREADS = 256;
+constexpr int EW_FLAT_ELEMS = 8192;      // elements per block on the flat path
+constexpr int EW_TILE = 64;              // transpose tile edge
+
+}  // namespace muon

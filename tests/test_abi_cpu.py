@@ -1,0 +1,164 @@
+"""The C-ABI library on the host: it builds, loads, exports every declared symbol,
+validates arguments without a GPU, and plans tile lists that cover every output
+element exactly once."""
+import ctypes
+import json
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import muon_newton_schulz_04_b200 as mb
+from muon_newton_schulz_04_b200 import build as mbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="session", autouse=True)
+def built_library():
+    mbuild.build()
+    return mb.lib()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "muon.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+\*?(muon_[a-z0-9_]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 18
+    L = ctypes.CDLL(mb.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(mb._SIGNATURES), set(names) ^ set(mb._SIGNATURES)
+
+
+def test_library_links_no_cuda_driver_at_load_time():
+    out = os.popen(f"ldd {mb.LIB_PATH}").read()
+    assert "libcuda.so" not in out
+    assert "libcudart" not in out          # runtime linked statically
+
+
+def test_default_config_matches_printed_coefficients():
+    g = json.load(open(os.path.join(ROOT, "tests", "golden", "ns_coefficients.json")))
+    c = mb.config()
+    assert (c.ns_a, c.ns_b, c.ns_c) == tuple(np.float32(v) for v in (g["a"], g["b"], g["c"]))
+    assert c.ns_steps == g["steps"] and c.nesterov == 1
+    assert abs(c.momentum - 0.95) < 1e-7 and abs(c.lr - 0.02) < 1e-9 and abs(c.eps - 1e-7) < 1e-13
+    assert mb.lib().muon_validate_config(ctypes.byref(c)) == mb.MUON_OK
+
+
+@pytest.mark.parametrize("field,value", [("momentum", 1.0), ("momentum", -0.1), ("ns_steps", -1), ("ns_steps", 17),
+                                         ("nesterov", 2), ("lr", float("nan")), ("weight_decay", -1.0),
+                                         ("eps", float("inf")), ("scale_mode", 7), ("precision", 3),
+                                         ("ns_a", float("inf"))])
+def test_config_validation_rejects(field, value):
+    c = mb.config()
+    setattr(c, field, value)
+    assert mb.lib().muon_validate_config(ctypes.byref(c)) == mb.MUON_ERR_INVALID
+
+
+def test_match_rms_needs_positive_target():
+    c = mb.config(scale_mode=mb.SCALE_MATCH_RMS, rms_target=0.0)
+    assert mb.lib().muon_validate_config(ctypes.byref(c)) == mb.MUON_ERR_INVALID
+    c = mb.config(scale_mode=mb.SCALE_MATCH_RMS, rms_target=0.2)
+    assert mb.lib().muon_validate_config(ctypes.byref(c)) == mb.MUON_OK
+
+
+def _group(rows=4, cols=8, count=2, dtype=mb.MUON_BF16, ptr=0x10000, w=None, g=None, b=None):
+    arrs = []
+    def mk(vals):
+        a = (ctypes.c_void_p * count)(*vals)
+        arrs.append(a)
+        return ctypes.cast(a, ctypes.POINTER(ctypes.c_void_p))
+    W = mk(w if w is not None else [ptr + 0x1000 * k for k in range(count)])
+    G = mk(g if g is not None else [ptr + 0x100000 + 0x1000 * k for k in range(count)])
+    B = mk(b if b is not None else [ptr + 0x200000 + 0x1000 * k for k in range(count)])
+    grp = mb._Group(rows, cols, count, dtype, 1.0, W, G, B)
+    return grp, arrs
+
+
+def test_group_validation():
+    L = mb.lib()
+    g, keep = _group()
+    assert L.muon_validate_groups(ctypes.byref(g), 1) == mb.MUON_OK
+    assert L.muon_validate_groups(None, 1) == mb.MUON_ERR_INVALID
+    assert L.muon_validate_groups(ctypes.byref(g), 0) == mb.MUON_ERR_INVALID
+    for kw in [dict(rows=0), dict(cols=-3), dict(count=0), dict(dtype=5),
+               dict(w=[0x10000, 0]), dict(b=[0x10000, 0x10002]), dict(g=[0x10001, 0x20000])]:
+        g2, keep2 = _group(**kw)
+        assert L.muon_validate_groups(ctypes.byref(g2), 1) == mb.MUON_ERR_INVALID, kw
+    g3, keep3 = _group(rows=1 << 16, cols=1 << 16)          # 2^32 elements
+    assert L.muon_validate_groups(ctypes.byref(g3), 1) == mb.MUON_ERR_INVALID
+    g4, keep4 = _group(dtype=mb.MUON_FP32, g=[0x10002, 0x20000])   # fp32 needs 4-byte alignment
+    assert L.muon_validate_groups(ctypes.byref(g4), 1) == mb.MUON_ERR_INVALID
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_create_without_gpu_reports_cuda_error():
+    h = ctypes.c_void_p()
+    c = mb.config()
+    st = mb.lib().muon_create(ctypes.byref(c), 0, ctypes.byref(h))
+    assert st in (mb.MUON_ERR_CUDA, mb.MUON_ERR_INVALID)
+    assert not h.value
+    assert mb.lib().muon_step(None, None, 0, None) == mb.MUON_ERR_INVALID
+    assert mb.lib().muon_destroy(None) == mb.MUON_ERR_INVALID
+
+
+def test_status_strings():
+    L = mb.lib()
+    assert L.muon_status_string(mb.MUON_OK) == b"MUON_OK"
+    assert L.muon_status_string(mb.MUON_ERR_DEVICE_TIMEOUT) == b"MUON_ERR_DEVICE_TIMEOUT"
+
+
+# ----------------------------------------------------------------------------- planner
+
+def _coverage(shapes, phase):
+    BM, BN = mb.tile_shape()
+    tiles = mb.plan_tiles(shapes, phase)
+    dims = [(min(r, c), max(r, c), k) for (r, c, k) in shapes]
+    cover = {}
+    for g, (m, n, k) in enumerate(dims):
+        cols = n if phase == 2 else m
+        cover[g] = np.zeros((k, m, cols), dtype=np.int32)
+    costs = []
+    for (g, z, ti, tj) in tiles:
+        m, n, k = dims[g]
+        costs.append(n if phase == 0 else m)
+        r0, c0 = ti * BM, tj * BN
+        rows = np.arange(r0, min(r0 + BM, m))
+        if phase == 2:
+            cols = np.arange(c0, min(c0 + BN, n))
+            cover[g][z][np.ix_(rows, cols)] += 1
+            continue
+        cols = np.arange(c0, min(c0 + BN, m))
+        R, C = np.meshgrid(rows, cols, indexing="ij")
+        direct = C >= R                      # the epilogue's store masks
+        mirror = C > R
+        np.add.at(cover[g][z], (R[direct], C[direct]), 1)
+        np.add.at(cover[g][z], (C[mirror], R[mirror]), 1)
+    return cover, costs
+
+
+@pytest.mark.parametrize("shapes", [[(256, 512, 1)], [(4096, 4096, 1)], [(768, 768, 4), (3072, 768, 1), (768, 3072, 1)],
+                                    [(1600, 1600, 2), (6400, 1600, 1)], [(37, 1000, 1), (1000, 37, 2)], [(1, 64, 1), (64, 1, 1)],
+                                    [(2048, 1408, 2), (16384, 4096, 1)]])
+@pytest.mark.parametrize("phase", [0, 1, 2])
+def test_tiles_cover_every_output_exactly_once(shapes, phase):
+    cover, costs = _coverage(shapes, phase)
+    for g, c in cover.items():
+        assert c.min() == 1 and c.max() == 1, (g, c.min(), c.max())
+    assert costs == sorted(costs, reverse=True)        # longest tiles first
+
+
+def test_symmetric_tiles_skip_the_lower_triangle():
+    BM, BN = mb.tile_shape()
+    full = len(mb.plan_tiles([(4096, 4096, 1)], 2))
+    sym = len(mb.plan_tiles([(4096, 4096, 1)], 0))
+    assert full == (4096 // BM) * (4096 // BN)
+    assert sym < 0.56 * full

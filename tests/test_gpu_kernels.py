@@ -1,0 +1,124 @@
+"""Per-kernel parity on the GPU: the three Newton-Schulz GEMMs (tensor-core bf16
+path and fp32 debug path) through muon_ns_phase_run, each against the oracle's
+piece of eq. 4 (gram, poly_matrix, ns_update) on the same bf16 inputs widened
+exactly to fp64.  Sizes span several 128x256 tiles with ragged tails."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import muon_newton_schulz_04_b200 as mb
+from muon_newton_schulz_04_b200 import build as mbuild
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def opt():
+    mbuild.build()
+    o = mb.Muon(mb.config())
+    yield o
+    o.close()
+
+
+def bf16(x: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).cuda()
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+SHAPES = [(128, 256, 1), (320, 776, 3), (384, 384, 2), (136, 1032, 1), (8, 64, 2), (520, 264, 1)]
+
+
+@pytest.mark.parametrize("m,n,count", SHAPES)
+def test_gram_bf16(opt, m, n, count):
+    rng = np.random.default_rng(m * 7 + n)
+    X = bf16(rng.standard_normal((count, m, n)) / np.sqrt(n))
+    out = torch.full((count, m, m), float("nan"), dtype=torch.bfloat16, device="cuda")
+    alpha = 0.75
+    opt.ns_phase(mb.NS_GRAM, mb.PREC_BF16, m, n, count, alpha, 0.0, x_op=X, out=out)
+    opt.sync()
+    Xh, A = f64(X), f64(out)
+    for z in range(count):
+        ref = alpha * oracle.gram(Xh[z])
+        bound = 2.0 ** -8 * np.abs(ref) + 1e-5 * alpha * (np.abs(Xh[z]) @ np.abs(Xh[z]).T)
+        assert np.all(np.abs(A[z] - ref) <= bound + 1e-30), float(np.max(np.abs(A[z] - ref) - bound))
+        assert np.array_equal(A[z], A[z].T)          # mirrored: exactly symmetric
+
+
+@pytest.mark.parametrize("m,n,count", SHAPES)
+def test_poly_bf16(opt, m, n, count):
+    rng = np.random.default_rng(m + 3 * n)
+    S = rng.standard_normal((count, m, m)) / np.sqrt(m)
+    S = S + np.transpose(S, (0, 2, 1))
+    A = bf16(S)
+    out = torch.full((count, m, m), float("nan"), dtype=torch.bfloat16, device="cuda")
+    a, b, c = oracle.NS_COEFFS
+    opt.ns_phase(mb.NS_POLY, mb.PREC_BF16, m, m, count, c, b, a_in=A, out=out)
+    opt.sync()
+    Ah, P = f64(A), f64(out)
+    for z in range(count):
+        ref = oracle.poly_matrix(Ah[z], b, c)
+        bound = 2.0 ** -8 * np.abs(ref) + 1e-5 * (abs(b) * np.abs(Ah[z]) + abs(c) * np.abs(Ah[z]) @ np.abs(Ah[z]))
+        assert np.all(np.abs(P[z] - ref) <= bound + 1e-30), float(np.max(np.abs(P[z] - ref) - bound))
+        assert np.array_equal(P[z], P[z].T)
+
+
+@pytest.mark.parametrize("m,n,count", SHAPES)
+def test_update_bf16(opt, m, n, count):
+    rng = np.random.default_rng(m + 5 * n)
+    P = bf16(rng.standard_normal((count, m, m)) / np.sqrt(m))
+    Xm = torch.from_numpy(rng.standard_normal((count, m, n)).astype(np.float32)).cuda()
+    Xop = Xm.to(torch.bfloat16)
+    out = torch.full((count, m, n), float("nan"), dtype=torch.float32, device="cuda")
+    out_op = torch.full((count, m, n), float("nan"), dtype=torch.bfloat16, device="cuda")
+    a = oracle.NS_COEFFS[0]
+    alpha = 1.25
+    opt.ns_phase(mb.NS_UPDATE, mb.PREC_BF16, m, n, count, alpha, a, x_op=Xop, a_in=P, x_master=Xm, out=out, out_op=out_op)
+    opt.sync()
+    Ph, Xh, Xmh, O = f64(P), f64(Xop), f64(Xm), f64(out)
+    for z in range(count):
+        # the GEMM reads the bf16 copy of X, the aX term the fp32 X
+        ref = alpha * (Ph[z] @ Xh[z]) + a * Xmh[z]
+        bound = 1e-5 * (abs(alpha) * np.abs(Ph[z]) @ np.abs(Xh[z]) + abs(a) * np.abs(Xmh[z])) + 1e-6 * np.abs(ref)
+        assert np.all(np.abs(O[z] - ref) <= bound), float(np.max(np.abs(O[z] - ref) - bound))
+        # the oracle's own step with the same operands agrees to bf16 input precision
+    assert torch.equal(out_op, out.to(torch.bfloat16))   # same rounding of the same fp32 value
+
+
+@pytest.mark.parametrize("m,n,count", [(64, 96, 2), (200, 136, 1), (37, 1000, 1)])
+def test_phases_fp32_debug(opt, m, n, count):
+    rng = np.random.default_rng(m * n)
+    X = torch.from_numpy(rng.standard_normal((count, m, n)).astype(np.float32)).cuda()
+    A = torch.empty(count, m, m, device="cuda")
+    opt.ns_phase(mb.NS_GRAM, mb.PREC_FP32_DEBUG, m, n, count, 0.5, 0.0, x_op=X, out=A)
+    P = torch.empty(count, m, m, device="cuda")
+    a, b, c = oracle.NS_COEFFS
+    opt.ns_phase(mb.NS_POLY, mb.PREC_FP32_DEBUG, m, m, count, c, b, a_in=A, out=P)
+    Y = torch.empty(count, m, n, device="cuda")
+    opt.ns_phase(mb.NS_UPDATE, mb.PREC_FP32_DEBUG, m, n, count, 1.0, a, x_op=X, a_in=P, x_master=X, out=Y)
+    opt.sync()
+    Xh = X.cpu().numpy().astype(np.float64)
+    for z in range(count):
+        Aref = 0.5 * oracle.gram(Xh[z])
+        assert np.max(np.abs(A[z].cpu().numpy() - Aref)) <= 1e-5 * np.max(np.abs(Aref)) * np.sqrt(n)
+        Pref = oracle.poly_matrix(A[z].cpu().numpy().astype(np.float64), b, c)
+        assert np.max(np.abs(P[z].cpu().numpy() - Pref)) <= 1e-5 * np.max(np.abs(Pref)) * np.sqrt(m)
+        Yref = oracle.ns_update(P[z].cpu().numpy().astype(np.float64), Xh[z], a)
+        assert np.max(np.abs(Y[z].cpu().numpy() - Yref)) <= 1e-5 * np.max(np.abs(Yref)) * np.sqrt(m)
+
+
+def test_phase_argument_errors(opt):
+    X = torch.zeros(1, 12, 16, dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros(1, 12, 12, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(mb.MuonError) as e:
+        opt.ns_phase(mb.NS_GRAM, mb.PREC_BF16, 12, 16, 1, 1.0, 0.0, x_op=X, out=out)   # m % 8 != 0
+    assert e.value.status == mb.MUON_ERR_UNSUPPORTED
+    with pytest.raises(mb.MuonError) as e:
+        opt.ns_phase(mb.NS_GRAM, mb.PREC_BF16, 16, 16, 1, 1.0, 0.0, x_op=None, out=out)
+    assert e.value.status == mb.MUON_ERR_INVALID
+    with pytest.raises(mb.MuonError) as e:
+        opt.ns_phase(7, mb.PREC_BF16, 16, 16, 1, 1.0, 0.0, x_op=X, out=out)
+    assert e.value.status == mb.MUON_ERR_INVALID
