@@ -240,6 +240,8 @@ def _map(fn, items: Sequence[int], threads: Optional[int]):
 
 def grads(wl: Workload, step: int, indices: Optional[Sequence[int]] = None, threads: Optional[int] = None):
     idx = list(range(wl.count)) if indices is None else list(indices)
+    if threads is None and wl.grad_kind in ("lowrank", "powerlaw"):
+        threads = 1          # QR-bound draws: the BLAS threads already use every core
     return _map(lambda k: grad(wl, step, k), idx, threads)
 
 
