@@ -199,6 +199,35 @@ muon_status muon_destroy(muon_handle* h);
 const char* muon_last_error(const muon_handle* h);
 const char* muon_status_string(muon_status s);
 
+/* ---- no-allocation entry point -----------------------------------------------
+ * The pages have no counterpart to this call.  It is for callers that cannot
+ * allocate device memory at all -- a runtime that owns a fixed device-memory pool
+ * and forbids allocations by anyone else, or code that runs while another
+ * component holds the allocator -- and so can use neither muon_create (which
+ * allocates an error word) nor the workspace of muon_step.
+ *
+ * It runs the momentum phase of ONE matrix (rows x cols, row-major, densely
+ * packed, device pointers on the current device): B <- momentum*B + G in place;
+ * the update direction U = G + momentum*B (nesterov = 1) or U = B (nesterov = 0)
+ * written to U_out (fp32, optional: NULL skips it); and ||U||_F written to
+ * norm_out (one float in device memory).  G is bf16 or fp32 (grad_dtype).
+ *
+ * It calls no cudaMalloc, cudaFree or other allocating routine and needs no
+ * handle.  Its only scratch, one fp64 partial sum per 8192 elements, is a static
+ * device array of MUON_NOALLOC_MAX_BLOCKS doubles (512 KiB) that every GPU which
+ * loads the library holds until the process exits; a matrix of more than
+ * MUON_NOALLOC_MAX_BLOCKS * 8192 elements is rejected with MUON_ERR_UNSUPPORTED.
+ * The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * All calls share the one array, and each call overwrites the partial sums it
+ * reads: calls whose work overlaps on the GPU (unordered streams) race and give
+ * wrong norms.  err_msg (optional host buffer of err_cap bytes) receives a
+ * message on failure. */
+#define MUON_NOALLOC_MAX_BLOCKS 65536
+muon_status muon_momentum_norm_noalloc(int rows, int cols, int grad_dtype, const void* G, float* B, float* U_out,
+                                       float momentum, int nesterov, float* norm_out, void* stream,
+                                       char* err_msg, int err_cap);
+
 /* ---- planner queries (host only, no GPU needed) ------------------------------
  * The persistent tensor-core GEMMs walk a tile list built once per shape set.
  * muon_plan_tiles writes the list a launch of `phase` would walk for the given

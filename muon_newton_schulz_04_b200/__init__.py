@@ -76,6 +76,9 @@ _SIGNATURES = {
     "muon_destroy": (ctypes.c_int, [ctypes.c_void_p]),
     "muon_last_error": (ctypes.c_char_p, [ctypes.c_void_p]),
     "muon_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "muon_momentum_norm_noalloc": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_int,
+                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int]),
     "muon_plan_tile_m": (ctypes.c_int, []),
     "muon_plan_tile_n": (ctypes.c_int, []),
     "muon_plan_tiles": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.c_int,
@@ -266,6 +269,21 @@ class Muon:
             self.close()
         except Exception:
             pass
+
+
+def momentum_norm_noalloc(G, B, norm_out, U_out=None, momentum: float = 0.95, nesterov: bool = True, stream=None):
+    """Momentum phase of one matrix with no device allocation (see muon.h):
+    B <- momentum*B + G in place, U_out = G + momentum*B (or B), norm_out[0] = ||U||_F."""
+    rows, cols = B.shape
+    _check_tensors([G, B], (rows, cols), True)
+    if U_out is not None:
+        _check_tensors([U_out], (rows, cols), True)
+    err = ctypes.create_string_buffer(256)
+    st = lib().muon_momentum_norm_noalloc(rows, cols, _dtype_code(G), G.data_ptr(), B.data_ptr(),
+                                          None if U_out is None else U_out.data_ptr(), float(momentum), int(nesterov),
+                                          norm_out.data_ptr(), ctypes.c_void_p(_stream(stream)), err, 256)
+    if st != MUON_OK:
+        raise MuonError(st, f"muon_momentum_norm_noalloc: {err.value.decode()}")
 
 
 def plan_tiles(shapes, phase: int):

@@ -21,7 +21,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libmuon_b200.so")
-SOURCES = ["api.cu", "elementwise.cu", "gemm_tc.cu", "gemm_simt.cu", "plan.cpp"]
+SOURCES = ["api.cu", "elementwise.cu", "gemm_tc.cu", "gemm_simt.cu", "plan.cpp", "noalloc.cu"]
 HEADERS = ["kernels.cuh", "ptx.cuh", "plan.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
