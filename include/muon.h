@@ -6,7 +6,7 @@
  * (papers.chlience.com synthesis note) defines it in section 4 "Muon 的算法定义":
  *
  *   B <- mu*B + G                                     (eq. 1, momentum)
- *   U <- G + mu*B   (Nesterov)   or   U <- B          (section 4: "Nesterov-style")
+ *   U <- G + mu*B   (Nesterov)   or   U <- B          (section 4: the Nesterov variant)
  *   X <- U, or U^T when rows > cols                   (section 4: smaller Gram)
  *   X <- X / (||X||_F + eps)                          (section 4: Frobenius normalisation)
  *   5 x  X <- aX + b(XX^T)X + c(XX^T)^2 X             (eqs. 4, 5: (a,b,c) = (3.4445,-4.7750,2.0315))
