@@ -326,6 +326,8 @@ def run_ours(args, w):
                    "shapes": sorted({f"{s.rows}x{s.cols}" for s in w.matrices}),
                    "ns_steps": w.ns_steps, "grad_dtype": w.grad_dtype, "weight_dtype": "fp32", "momentum_dtype": "fp32",
                    "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "gemm": "tcgen05 cta_group::2, 256x256 tiles" if os.environ.get("MUON_GEMM_PAIR", "1") != "0"
+                           else "tcgen05 cta_group::1, 128x256 tiles",
                    "l2": f"working set {ws_bytes / 2**20:.0f} MiB > 126 MiB L2 (no flush)",
                    "flops_per_step_nominal": flops_nom, "flops_per_step_symmetric": w.ns_flops_symmetric()},
         "ns5_tflops": round(ns_tflops, 2),
@@ -335,7 +337,7 @@ def run_ours(args, w):
         "apply_gbs": round(b_app / (app_ms * 1e-3) / 1e9, 1),
         "apply_frac_of_hbm": round(b_app / (app_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
         "phase_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
-        "roofline": {"kernel": "ns_gemm_tc_kernel<UPDATE> (X' = P X + aX)", "bound": "tensor",
+        "roofline": {"kernel": "update GEMM X' = P X + aX (ns_gemm_tc2_kernel<2>)", "bound": "tensor",
                      "achieved": round(upd_tflops, 2), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(upd_tflops / peaks["bf16_tflops"], 4), "traffic": None,
                      "peak_source": f"{peak_src} bf16 dense (burst)",

@@ -66,6 +66,8 @@ struct muon_handle {
     muon_config cfg;
     int device = 0;
     int num_sms = 148;
+    int pair = 1;            // 1: two-CTA GEMM kernel, 0: one-CTA kernel
+    int max_clusters = 74;   // co-resident two-CTA clusters of the pair kernel
     std::string last_error;
     DevBuf ws;            // plan workspace
     DevBuf staging;       // muon_step_host staging
@@ -248,6 +250,12 @@ muon_status encode_map(muon_handle* h, CUtensorMap* m, const void* base, int col
 
 bool is_bf16_path(const muon_handle* h) { return h->cfg.precision == MUON_PREC_BF16; }
 
+// Persistent grid: one CTA (or one two-CTA cluster) per tile, at most one per SM.
+int gemm_grid(const muon_handle* h, int ntiles) {
+    if (h->pair) return 2 * std::min(ntiles, h->max_clusters);
+    return std::min(ntiles, h->num_sms);
+}
+
 // Builds (or reuses) the plan for the shape list; allocates the workspace,
 // writes tile lists, tensor maps and group descriptors to the device.
 muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStream_t s) {
@@ -295,9 +303,10 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
     P.k7_blocks = k7;
     std::vector<Tile> tg, tp, tu;
     if (bf16) {
-        tg = build_tiles(P.dims, 0, TC_BM, TC_BN);
-        tp = build_tiles(P.dims, 1, TC_BM, TC_BN);
-        tu = build_tiles(P.dims, 2, TC_BM, TC_BN);
+        const int bm = tc_gemm_tile_m(h->pair), bn = tc_gemm_tile_n(h->pair);
+        tg = build_tiles(P.dims, 0, bm, bn);
+        tp = build_tiles(P.dims, 1, bm, bn);
+        tu = build_tiles(P.dims, 2, bm, bn);
     }
     P.n_gram = (int)tg.size(); P.n_poly = (int)tp.size(); P.n_upd = (int)tu.size();
     const size_t o_tg = take(tg.size() * sizeof(int4) + 16), o_tp = take(tp.size() * sizeof(int4) + 16),
@@ -366,6 +375,8 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
         CUDA_TRY(h, cudaStreamSynchronize(s));
         if (!h->tc_ready) {
             CUDA_TRY(h, tc_gemm_prepare());
+            CUDA_TRY(h, tc_gemm_max_clusters(&h->max_clusters));
+            if (h->max_clusters < 1) return fail(h, MUON_ERR_UNSUPPORTED, "no two-CTA cluster fits on this device");
             h->tc_ready = true;
         }
     }
@@ -426,13 +437,13 @@ muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStrea
             gp.maps = P.d_maps; gp.groups = P.d_ginfo; gp.parity = par; gp.err = h->d_err;
             gp.tiles = P.d_tiles_gram; gp.ntiles = P.n_gram; gp.alpha = 1.f; gp.beta = 0.f;
             gp.scale = it == 0 ? P.d_scale : nullptr;
-            TIMED(h, 2, s, launch_tc_gemm(MODE_GRAM, gp, std::min(P.n_gram, h->num_sms), s));
+            TIMED(h, 2, s, launch_tc_gemm(MODE_GRAM, h->pair, gp, gemm_grid(h, P.n_gram), s));
             gp.tiles = P.d_tiles_poly; gp.ntiles = P.n_poly; gp.alpha = c.ns_c; gp.beta = c.ns_b; gp.scale = nullptr;
-            TIMED(h, 3, s, launch_tc_gemm(MODE_POLY, gp, std::min(P.n_poly, h->num_sms), s));
+            TIMED(h, 3, s, launch_tc_gemm(MODE_POLY, h->pair, gp, gemm_grid(h, P.n_poly), s));
             gp.tiles = P.d_tiles_upd; gp.ntiles = P.n_upd; gp.alpha = 1.f; gp.beta = c.ns_a;
             gp.scale = it == 0 ? P.d_scale : nullptr;
             gp.write_op = (it + 1 < c.ns_steps) ? 1 : 0;
-            TIMED(h, 4, s, launch_tc_gemm(MODE_UPDATE, gp, std::min(P.n_upd, h->num_sms), s));
+            TIMED(h, 4, s, launch_tc_gemm(MODE_UPDATE, h->pair, gp, gemm_grid(h, P.n_upd), s));
         } else {
             for (size_t g = 0; g < P.dims.size(); ++g) {
                 const GroupDims& d = P.dims[g];
@@ -533,6 +544,7 @@ muon_status muon_create(const muon_config* cfg, int device, muon_handle** out) {
     h->cfg = *cfg;
     h->device = device;
     h->num_sms = prop.multiProcessorCount;
+    h->pair = tc_gemm_default_pair();
     DeviceGuard dg(device);
     if (cudaMalloc(&h->d_err, sizeof(int)) != cudaSuccess || cudaMemset(h->d_err, 0, sizeof(int)) != cudaSuccess) {
         cudaGetLastError();
@@ -684,12 +696,18 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     }
     muon_status st = load_encoder(h);
     if (st != MUON_OK) return st;
-    if (!h->tc_ready) { CUDA_TRY(h, tc_gemm_prepare()); h->tc_ready = true; }
+    if (!h->tc_ready) {
+        CUDA_TRY(h, tc_gemm_prepare());
+        CUDA_TRY(h, tc_gemm_max_clusters(&h->max_clusters));
+        if (h->max_clusters < 1) return fail(h, MUON_ERR_UNSUPPORTED, "no two-CTA cluster fits on this device");
+        h->tc_ready = true;
+    }
     GroupDims d{};
     d.rows = m; d.cols = n; d.count = cnt; d.m = m; d.n = n; d.ldm = m; d.ldn = n; d.transposed = 0;
     std::vector<GroupDims> dims(1, d);
     const int phase = a->phase;
-    std::vector<Tile> tl = build_tiles(dims, phase == MUON_NS_UPDATE ? 2 : phase, TC_BM, TC_BN);
+    std::vector<Tile> tl = build_tiles(dims, phase == MUON_NS_UPDATE ? 2 : phase, tc_gemm_tile_m(h->pair),
+                                       tc_gemm_tile_n(h->pair));
     GemmMaps maps{};
     GemmGroupInfo gi{};
     gi.m = m; gi.n = n; gi.ldm = m; gi.ldn = n; gi.count = cnt; gi.mat_base = 0;
@@ -731,7 +749,7 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     gp.write_op = (phase == MUON_NS_UPDATE && a->out_op) ? 1 : 0;
     gp.err = h->d_err;
     const int mode = phase == MUON_NS_GRAM ? MODE_GRAM : phase == MUON_NS_POLY ? MODE_POLY : MODE_UPDATE;
-    CUDA_TRY(h, launch_tc_gemm(mode, gp, std::min(gp.ntiles, h->num_sms), s));
+    CUDA_TRY(h, launch_tc_gemm(mode, h->pair, gp, gemm_grid(h, gp.ntiles), s));
     return MUON_OK;
 }
 
@@ -830,8 +848,8 @@ const char* muon_status_string(muon_status s) {
     return "unknown status";
 }
 
-int muon_plan_tile_m(void) { return TC_BM; }
-int muon_plan_tile_n(void) { return TC_BN; }
+int muon_plan_tile_m(void) { return tc_gemm_tile_m(tc_gemm_default_pair()); }
+int muon_plan_tile_n(void) { return tc_gemm_tile_n(tc_gemm_default_pair()); }
 
 muon_status muon_plan_tiles(const int* shapes, int n_groups, int phase, int* out, int cap, int* n_tiles) {
     if (!shapes || n_groups <= 0 || !n_tiles || phase < 0 || phase > 2) return MUON_ERR_INVALID;
@@ -841,7 +859,8 @@ muon_status muon_plan_tiles(const int* shapes, int n_groups, int phase, int* out
         if (check_shape(shapes[3 * g], shapes[3 * g + 1], shapes[3 * g + 2], &why) != MUON_OK) return MUON_ERR_INVALID;
         dims.push_back(make_dims(shapes[3 * g], shapes[3 * g + 1], shapes[3 * g + 2]));
     }
-    std::vector<Tile> t = build_tiles(dims, phase, TC_BM, TC_BN);
+    const int pair = tc_gemm_default_pair();
+    std::vector<Tile> t = build_tiles(dims, phase, tc_gemm_tile_m(pair), tc_gemm_tile_n(pair));
     *n_tiles = (int)t.size();
     if (!out || cap < (int)t.size()) return MUON_ERR_INVALID;
     for (size_t i = 0; i < t.size(); ++i) {

@@ -11,37 +11,54 @@
 // On the first step alpha/beta absorb the Frobenius normalisation s = 1/(||U||+eps):
 // A0 = s^2 UU^T and X1 = s P U + a s U.
 //
-// Kernel structure (one CTA per SM, 320 threads):
+// Two kernels share the epilogue:
+//
+//  ns_gemm_tc_kernel (one CTA per tile, 128 x 256 tiles), 320 threads:
 //   warp 0      TMA producer: 4-stage ring of (128x64 A-operand, 256x64 B-operand)
-//               bf16 tiles in 128-byte-swizzled shared memory, plain (non-multicast)
-//               3-D tiled loads, zero fill outside the matrix.
-//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators) and
-//               issues tcgen05.mma kind::f16 (M=128, N=256, K=16) from one thread;
-//               tcgen05.commit frees ring slots and publishes finished accumulators.
+//               bf16 tiles in 128-byte-swizzled shared memory, plain 3-D tiled loads.
+//   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators) and issues
+//               tcgen05.mma kind::f16 (M=128, N=256, K=16) from one thread.
 //   warps 2-9   epilogue: tcgen05.ld of the accumulator (each warp owns the 32 TMEM
-//               lanes its rank allows and half of the columns), scale, add the
-//               residual term, round, store; mirrored stores for the symmetric outputs.
-// The double-buffered accumulator lets the epilogue of tile i overlap the
-// main loop of tile i+1.  Tiles are taken round-robin from a cost-sorted list
-// that spans all matrices of the call, so many small matrices fill the 148 SMs.
+//               lanes its rank allows and half of the columns), scale, residual, store.
+//
+//  ns_gemm_tc2_kernel (a cluster of two CTAs per 256 x 256 tile): each CTA stages its
+//   128 rows of A and its 128 columns of B (6-stage ring of 16 + 16 KiB), the even CTA
+//   issues tcgen05.mma.cta_group::2 (M=256, N=256) which reads both CTAs' shared memory,
+//   and each CTA's TMEM receives its 128 accumulator rows.  Per SM this moves half the
+//   B-operand bytes of the one-CTA tile through shared memory.  The odd CTA's TMA
+//   loads complete on the even CTA's barrier; MMA completion is committed to the
+//   barriers of both CTAs by address; no multicast form is used.
+//
+// The double-buffered accumulator lets the epilogue of tile i overlap the main
+// loop of tile i+1.  Tiles are taken round-robin from a cost-sorted list that
+// spans all matrices of the call, so many small matrices fill the 148 SMs.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
 namespace muon {
 namespace {
 
-constexpr int BM = TC_BM, BN = TC_BN, BK = TC_BK;
-constexpr int STAGES = 4;
-constexpr int A_STAGE = BM * BK * 2;      // 16 KiB
-constexpr int B_STAGE = BN * BK * 2;      // 32 KiB
-constexpr int STAGE_BYTES = A_STAGE + B_STAGE;
+constexpr int BK = TC_BK;
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
-constexpr int TMEM_COLS = 2 * BN;          // two accumulators
-constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/;
+constexpr int ACC_COLS = 256;                 // one accumulator: 128 lanes x 256 fp32 columns
+constexpr int TMEM_COLS = 2 * ACC_COLS;       // two accumulators
+
+// one-CTA kernel
+constexpr int S1_BM = 128, S1_BN = 256, S1_STAGES = 4;
+constexpr int S1_A = S1_BM * BK * 2;          // 16 KiB
+constexpr int S1_B = S1_BN * BK * 2;          // 32 KiB
+constexpr int S1_SMEM = 1024 + S1_STAGES * (S1_A + S1_B) + 256;
+
+// two-CTA kernel (per CTA)
+constexpr int S2_BM = 256, S2_BN = 256, S2_STAGES = 6;
+constexpr int S2_A = 128 * BK * 2;            // 16 KiB: this CTA's 128 rows of A
+constexpr int S2_B = 128 * BK * 2;            // 16 KiB: this CTA's 128 columns of B
+constexpr int S2_SMEM = 1024 + S2_STAGES * (S2_A + S2_B) + 256;
 
 // error codes written to the device error word when a bounded wait gives up
-constexpr int ERR_PRODUCER = 0x101, ERR_MMA_SLOT = 0x102, ERR_MMA_ACC = 0x103, ERR_EPILOGUE = 0x104;
+constexpr int ERR_PRODUCER = 0x101, ERR_MMA_SLOT = 0x102, ERR_MMA_ACC = 0x103, ERR_EPILOGUE = 0x104,
+              ERR_TAIL = 0x105;
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -51,8 +68,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_bits_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_bits_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Epilogue of one 32-column chunk of one output row for the symmetric outputs
-// (GRAM and POLY).  val[] holds the finished fp32 values of columns col0..col0+31.
+// Stores one 32-column chunk of one output row of a symmetric output (GRAM, POLY).
 // Element (row, c) is stored directly when c >= row and mirrored to (c, row) when
 // c > row, so every element of the m x m output is written exactly once.
 __device__ __forceinline__ void store_symmetric(__nv_bfloat16* __restrict__ out, int m, int ldm,
@@ -85,15 +101,127 @@ __device__ __forceinline__ void store_symmetric(__nv_bfloat16* __restrict__ out,
     }
 }
 
+// Epilogue of one accumulator row segment: 4 chunks of 32 columns starting at
+// column `c_begin` of the accumulator whose TMEM address (lane quarter included)
+// is `tacc`.  `row` is the global output row of this thread, `col_base` the
+// global column of accumulator column 0.
+template <int MODE>
+__device__ __forceinline__ void epilogue_segment(const GemmParams& p, const GemmGroupInfo& gi, int mat, int row,
+                                                 int col_base, uint32_t tacc, int c_begin) {
+    float alpha = p.alpha, beta = p.beta;
+    if (p.scale != nullptr) {
+        const float s = p.scale[gi.mat_base + mat];
+        if (MODE == MODE_GRAM) alpha = p.alpha * s * s;
+        if (MODE == MODE_UPDATE) { alpha = p.alpha * s; beta = p.beta * s; }
+    }
+#pragma unroll 1
+    for (int chunk = 0; chunk < 4; ++chunk) {
+        const int c_local = c_begin + chunk * 32;
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tacc + (uint32_t)c_local, v);
+        tmem_ld_wait();
+        const int col0 = col_base + c_local;
+        float val[32];
+        if (MODE == MODE_GRAM) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) val[j] = alpha * __uint_as_float(v[j]);
+            store_symmetric(gi.a + (size_t)mat * gi.m * gi.ldm, gi.m, gi.ldm, row, col0, val);
+        } else if (MODE == MODE_POLY) {
+            const __nv_bfloat16* A = gi.a + (size_t)mat * gi.m * gi.ldm;
+            if (row < gi.m && col0 + 31 < gi.m) {
+                const uint4* src = reinterpret_cast<const uint4*>(A + (size_t)row * gi.ldm + col0);
+#pragma unroll
+                for (int qq = 0; qq < 4; ++qq) {
+                    const uint4 w = src[qq];
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        val[8 * qq + 2 * e] = alpha * __uint_as_float(v[8 * qq + 2 * e]) + beta * bf16_bits_lo(ws[e]);
+                        val[8 * qq + 2 * e + 1] = alpha * __uint_as_float(v[8 * qq + 2 * e + 1]) + beta * bf16_bits_hi(ws[e]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int c = col0 + j;
+                    const float av = (row < gi.m && c < gi.m) ? __bfloat162float(A[(size_t)row * gi.ldm + c]) : 0.f;
+                    val[j] = alpha * __uint_as_float(v[j]) + beta * av;
+                }
+            }
+            store_symmetric(gi.p + (size_t)mat * gi.m * gi.ldm, gi.m, gi.ldm, row, col0, val);
+        } else {
+            if (row < gi.m) {
+                const size_t off = (size_t)mat * gi.m * gi.ldn + (size_t)row * gi.ldn;
+                const float* xin = gi.xf_in + off;
+                float* xout = gi.xf_out + off;
+                __nv_bfloat16* xb = gi.xb[p.parity ^ 1] + off;
+                if (col0 + 31 < gi.n) {
+                    const float4* src = reinterpret_cast<const float4*>(xin + col0);
+#pragma unroll
+                    for (int qq = 0; qq < 8; ++qq) {
+                        const float4 x = src[qq];
+                        val[4 * qq + 0] = alpha * __uint_as_float(v[4 * qq + 0]) + beta * x.x;
+                        val[4 * qq + 1] = alpha * __uint_as_float(v[4 * qq + 1]) + beta * x.y;
+                        val[4 * qq + 2] = alpha * __uint_as_float(v[4 * qq + 2]) + beta * x.z;
+                        val[4 * qq + 3] = alpha * __uint_as_float(v[4 * qq + 3]) + beta * x.w;
+                    }
+                    float4* dst = reinterpret_cast<float4*>(xout + col0);
+#pragma unroll
+                    for (int qq = 0; qq < 8; ++qq)
+                        dst[qq] = make_float4(val[4 * qq], val[4 * qq + 1], val[4 * qq + 2], val[4 * qq + 3]);
+                    if (p.write_op) {
+                        uint4* db = reinterpret_cast<uint4*>(xb + col0);
+#pragma unroll
+                        for (int qq = 0; qq < 4; ++qq) {
+                            uint4 w;
+                            w.x = pack_bf16x2(val[8 * qq + 0], val[8 * qq + 1]);
+                            w.y = pack_bf16x2(val[8 * qq + 2], val[8 * qq + 3]);
+                            w.z = pack_bf16x2(val[8 * qq + 4], val[8 * qq + 5]);
+                            w.w = pack_bf16x2(val[8 * qq + 6], val[8 * qq + 7]);
+                            db[qq] = w;
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const int c = col0 + j;
+                        if (c < gi.n) {
+                            const float r = alpha * __uint_as_float(v[j]) + beta * xin[c];
+                            xout[c] = r;
+                            if (p.write_op) xb[c] = __float2bfloat16_rn(r);
+                        }
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int MODE>
+__device__ __forceinline__ void operand_maps(const GemmParams& p, int g, const void*& mapA, const void*& mapB) {
+    const GemmMaps* mp = p.maps + g;
+    mapA = (MODE == MODE_GRAM) ? (const void*)&mp->xb_k[p.parity]
+         : (MODE == MODE_POLY) ? (const void*)&mp->a : (const void*)&mp->p;
+    mapB = (MODE == MODE_GRAM) ? (const void*)&mp->xb_k[p.parity]
+         : (MODE == MODE_POLY) ? (const void*)&mp->a : (const void*)&mp->xb_mn[p.parity];
+}
+
+__device__ __forceinline__ void spin_ns(uint64_t ns) {
+    const uint64_t t0 = globaltimer_ns();
+    while (globaltimer_ns() - t0 < ns) { }
+}
+
+// ============================================================================ one-CTA kernel
+
 template <int MODE>
 __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid_constant__ GemmParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + STAGES * A_STAGE;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
-    uint64_t* empty = full + STAGES;
-    uint64_t* tfull = empty + STAGES;
+    uint8_t* sB = smem + S1_STAGES * S1_A;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S1_STAGES * (S1_A + S1_B));
+    uint64_t* empty = full + S1_STAGES;
+    uint64_t* tfull = empty + S1_STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -103,7 +231,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid
     const uint32_t lane = threadIdx.x & 31u;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < S1_STAGES; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
@@ -125,30 +253,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid
     const uint32_t tmem_base = *tmem_slot;
 
     if (warp == 0) {
-        // ------------------------------------------------------------ TMA producer
         if (elect_one()) {
             uint32_t stage = 0, phase = 0;
             bool ok = true;
             for (int t = blockIdx.x; t < p.ntiles && ok; t += gridDim.x) {
                 const int4 tile = p.tiles[t];
                 const GemmGroupInfo& gi = p.groups[tile.x];
-                const GemmMaps* mp = p.maps + tile.x;
                 const int K = (MODE == MODE_GRAM) ? gi.n : gi.m;
                 const int kblocks = (K + BK - 1) / BK;
-                const void* mapA = (MODE == MODE_GRAM) ? (const void*)&mp->xb_k[p.parity]
-                                 : (MODE == MODE_POLY) ? (const void*)&mp->a : (const void*)&mp->p;
-                const void* mapB = (MODE == MODE_GRAM) ? (const void*)&mp->xb_k[p.parity]
-                                 : (MODE == MODE_POLY) ? (const void*)&mp->a : (const void*)&mp->xb_mn[p.parity];
-                const int row0 = tile.z * BM, col0 = tile.w * BN, mat = tile.y;
+                const void *mapA, *mapB;
+                operand_maps<MODE>(p, tile.x, mapA, mapB);
+                const int row0 = tile.z * S1_BM, col0 = tile.w * S1_BN, mat = tile.y;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, ERR_PRODUCER)) { ok = false; break; }
-                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                    mbar_arrive_expect_tx(&full[stage], S1_A + S1_B);
                     const int k0 = kb * BK;
-                    uint8_t* a_dst = sA + stage * A_STAGE;
-                    uint8_t* b_dst = sB + stage * B_STAGE;
+                    uint8_t* a_dst = sA + stage * S1_A;
+                    uint8_t* b_dst = sB + stage * S1_B;
                     tma_load_3d(a_dst, mapA, &full[stage], k0, row0, mat);
                     if (MODE == MODE_UPDATE) {
-                        // B = X rows k0..k0+63, columns col0..col0+255, as four 64-column boxes
 #pragma unroll
                         for (int c = 0; c < 4; ++c)
                             tma_load_3d(b_dst + c * (BK * 128), mapB, &full[stage], col0 + 64 * c, k0, mat);
@@ -156,19 +279,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid
                         tma_load_3d(b_dst, mapB, &full[stage], k0, col0, mat);
                         tma_load_3d(b_dst + 128 * 128, mapB, &full[stage], k0, col0 + 128, mat);
                     }
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    if (++stage == S1_STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            if (!ok || *abort_flag) {
-                // let any load still in flight land before the CTA retires
-                const uint64_t t0 = globaltimer_ns();
-                while (globaltimer_ns() - t0 < 2000000ull) { }
+            // tail: every slot released once more, so no MMA completion is still
+            // on its way to this CTA's barriers when it retires
+            for (int i = 0; i < S1_STAGES && ok; ++i) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, ERR_TAIL)) ok = false;
+                if (++stage == S1_STAGES) { stage = 0; phase ^= 1u; }
             }
+            if (!ok || *abort_flag) spin_ns(2000000ull);   // let loads in flight land
         }
     } else if (warp == 1) {
-        // ------------------------------------------------------------ MMA issuer
         if (elect_one()) {
-            constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, MODE == MODE_UPDATE ? 1u : 0u);
+            constexpr uint32_t idesc = idesc_bf16_f32(S1_BM, S1_BN, MODE == MODE_UPDATE ? 1u : 0u);
             uint32_t stage = 0, phase = 0;
             int local = 0;
             bool ok = true;
@@ -181,12 +305,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid
                 const uint32_t acc_phase = (local >> 1) & 1;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.err, ERR_MMA_ACC)) { ok = false; break; }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + acc * BN;
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag, p.err, ERR_MMA_SLOT)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a_base = smem_u32(sA + stage * A_STAGE);
-                    const uint32_t b_base = smem_u32(sB + stage * B_STAGE);
+                    const uint32_t a_base = smem_u32(sA + stage * S1_A);
+                    const uint32_t b_base = smem_u32(sB + stage * S1_B);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         // K-major 128B-swizzled: rows 128 B apart, 8-row groups 1024 B apart;
@@ -203,22 +327,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid
                         tc_mma_f16(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit(&empty[stage]);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                    if (++stage == S1_STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 tc_commit(&tfull[acc]);
             }
             if (!ok || *abort_flag) {
-                // wait (bounded) until every MMA issued so far has finished
                 tc_commit(drain);
                 const uint64_t t0 = globaltimer_ns();
                 while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 100000000ull) { }
             }
         }
     } else {
-        // ------------------------------------------------------------ epilogue
-        const uint32_t q = warp & 3u;                 // TMEM lane quarter this warp may access
-        const uint32_t half = (warp - 2) >> 2;        // column half of the tile
+        const uint32_t q = warp & 3u;
+        const uint32_t half = (warp - 2) >> 2;
         int local = 0;
         for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++local) {
             const int4 tile = p.tiles[t];
@@ -228,96 +350,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid
             bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, ERR_EPILOGUE);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-
-            const int mat = tile.y;
-            const int row = tile.z * BM + (int)(q * 32 + lane);
-            float alpha = p.alpha, beta = p.beta;
-            if (p.scale != nullptr) {
-                const float s = p.scale[gi.mat_base + mat];
-                if (MODE == MODE_GRAM) alpha = p.alpha * s * s;
-                if (MODE == MODE_UPDATE) { alpha = p.alpha * s; beta = p.beta * s; }
-            }
-#pragma unroll 1
-            for (int chunk = 0; chunk < 4; ++chunk) {
-                const int c_local = (int)half * 128 + chunk * 32;
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tmem_base + acc * BN + ((q * 32u) << 16) + (uint32_t)c_local, v);
-                tmem_ld_wait();
-                const int col0 = tile.w * BN + c_local;
-                float val[32];
-                if (MODE == MODE_GRAM) {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) val[j] = alpha * __uint_as_float(v[j]);
-                    store_symmetric(gi.a + (size_t)mat * gi.m * gi.ldm, gi.m, gi.ldm, row, col0, val);
-                } else if (MODE == MODE_POLY) {
-                    const __nv_bfloat16* A = gi.a + (size_t)mat * gi.m * gi.ldm;
-                    if (row < gi.m && col0 + 31 < gi.m) {
-                        const uint4* src = reinterpret_cast<const uint4*>(A + (size_t)row * gi.ldm + col0);
-#pragma unroll
-                        for (int qq = 0; qq < 4; ++qq) {
-                            const uint4 w = src[qq];
-                            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                            for (int e = 0; e < 4; ++e) {
-                                val[8 * qq + 2 * e] = alpha * __uint_as_float(v[8 * qq + 2 * e]) + beta * bf16_bits_lo(ws[e]);
-                                val[8 * qq + 2 * e + 1] = alpha * __uint_as_float(v[8 * qq + 2 * e + 1]) + beta * bf16_bits_hi(ws[e]);
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j) {
-                            const int c = col0 + j;
-                            const float av = (row < gi.m && c < gi.m) ? __bfloat162float(A[(size_t)row * gi.ldm + c]) : 0.f;
-                            val[j] = alpha * __uint_as_float(v[j]) + beta * av;
-                        }
-                    }
-                    store_symmetric(gi.p + (size_t)mat * gi.m * gi.ldm, gi.m, gi.ldm, row, col0, val);
-                } else {
-                    if (row < gi.m) {
-                        const size_t off = (size_t)mat * gi.m * gi.ldn + (size_t)row * gi.ldn;
-                        const float* xin = gi.xf_in + off;
-                        float* xout = gi.xf_out + off;
-                        __nv_bfloat16* xb = gi.xb[p.parity ^ 1] + off;
-                        if (col0 + 31 < gi.n) {
-                            const float4* src = reinterpret_cast<const float4*>(xin + col0);
-#pragma unroll
-                            for (int qq = 0; qq < 8; ++qq) {
-                                const float4 x = src[qq];
-                                val[4 * qq + 0] = alpha * __uint_as_float(v[4 * qq + 0]) + beta * x.x;
-                                val[4 * qq + 1] = alpha * __uint_as_float(v[4 * qq + 1]) + beta * x.y;
-                                val[4 * qq + 2] = alpha * __uint_as_float(v[4 * qq + 2]) + beta * x.z;
-                                val[4 * qq + 3] = alpha * __uint_as_float(v[4 * qq + 3]) + beta * x.w;
-                            }
-                            float4* dst = reinterpret_cast<float4*>(xout + col0);
-#pragma unroll
-                            for (int qq = 0; qq < 8; ++qq)
-                                dst[qq] = make_float4(val[4 * qq], val[4 * qq + 1], val[4 * qq + 2], val[4 * qq + 3]);
-                            if (p.write_op) {
-                                uint4* db = reinterpret_cast<uint4*>(xb + col0);
-#pragma unroll
-                                for (int qq = 0; qq < 4; ++qq) {
-                                    uint4 w;
-                                    w.x = pack_bf16x2(val[8 * qq + 0], val[8 * qq + 1]);
-                                    w.y = pack_bf16x2(val[8 * qq + 2], val[8 * qq + 3]);
-                                    w.z = pack_bf16x2(val[8 * qq + 4], val[8 * qq + 5]);
-                                    w.w = pack_bf16x2(val[8 * qq + 6], val[8 * qq + 7]);
-                                    db[qq] = w;
-                                }
-                            }
-                        } else {
-#pragma unroll
-                            for (int j = 0; j < 32; ++j) {
-                                const int c = col0 + j;
-                                if (c < gi.n) {
-                                    const float r = alpha * __uint_as_float(v[j]) + beta * xin[c];
-                                    xout[c] = r;
-                                    if (p.write_op) xb[c] = __float2bfloat16_rn(r);
-                                }
-                            }
-                        }
-                    }
-                }
-            }
+            const int row = tile.z * S1_BM + (int)(q * 32 + lane);
+            epilogue_segment<MODE>(p, gi, tile.y, row, tile.w * S1_BN,
+                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * 128);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -332,24 +367,208 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid
     }
 }
 
+// ============================================================================ two-CTA kernel
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + S2_STAGES * S2_A;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S2_STAGES * (S2_A + S2_B));
+    uint64_t* empty = full + S2_STAGES;
+    uint64_t* tfull = empty + S2_STAGES;
+    uint64_t* tempty = tfull + 2;
+    uint64_t* drain = tempty + 2;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const uint32_t warp = warp_id();
+    const uint32_t lane = threadIdx.x & 31u;
+    const uint32_t rank = cluster_ctarank();          // 0: issues the MMA
+    const int cid = (int)cluster_id_x();
+    const int ncl = (int)nclusters_x();
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S2_STAGES; ++s) {
+            mbar_init(&full[s], 1);                   // used in CTA 0: its producer's arrive + both CTAs' bytes
+            mbar_init(&empty[s], 1);                  // one commit from the MMA thread
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull[b], 1);
+            mbar_init(&tempty[b], 2 * NUM_EPI_WARPS); // used in CTA 0: epilogue warps of both CTAs
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync_all();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        if (elect_one()) {
+            uint32_t stage = 0, phase = 0;
+            bool ok = true;
+            for (int t = cid; t < p.ntiles && ok; t += ncl) {
+                const int4 tile = p.tiles[t];
+                const GemmGroupInfo& gi = p.groups[tile.x];
+                const int K = (MODE == MODE_GRAM) ? gi.n : gi.m;
+                const int kblocks = (K + BK - 1) / BK;
+                const void *mapA, *mapB;
+                operand_maps<MODE>(p, tile.x, mapA, mapB);
+                const int row0 = tile.z * S2_BM + (int)rank * 128;     // this CTA's rows of A
+                const int colh = tile.w * S2_BN + (int)rank * 128;     // this CTA's columns of B
+                const int mat = tile.y;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, ERR_PRODUCER)) { ok = false; break; }
+                    const uint32_t full0 = mapa_shared(smem_u32(&full[stage]), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (S2_A + S2_B));
+                    const int k0 = kb * BK;
+                    uint8_t* a_dst = sA + stage * S2_A;
+                    uint8_t* b_dst = sB + stage * S2_B;
+                    tma_load_3d_pair(a_dst, mapA, full0, k0, row0, mat);
+                    if (MODE == MODE_UPDATE) {
+                        tma_load_3d_pair(b_dst, mapB, full0, colh, k0, mat);
+                        tma_load_3d_pair(b_dst + BK * 128, mapB, full0, colh + 64, k0, mat);
+                    } else {
+                        tma_load_3d_pair(b_dst, mapB, full0, k0, colh, mat);
+                    }
+                    if (++stage == S2_STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            for (int i = 0; i < S2_STAGES && ok; ++i) {
+                if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, ERR_TAIL)) ok = false;
+                if (++stage == S2_STAGES) { stage = 0; phase ^= 1u; }
+            }
+            if (!ok || *abort_flag) spin_ns(2000000ull);
+        }
+    } else if (warp == 1) {
+        if (rank == 0 && elect_one()) {
+            constexpr uint32_t idesc = idesc_bf16_f32(S2_BM, S2_BN, MODE == MODE_UPDATE ? 1u : 0u);
+            uint32_t stage = 0, phase = 0;
+            int local = 0;
+            bool ok = true;
+            for (int t = cid; t < p.ntiles && ok; t += ncl, ++local) {
+                const int4 tile = p.tiles[t];
+                const GemmGroupInfo& gi = p.groups[tile.x];
+                const int K = (MODE == MODE_GRAM) ? gi.n : gi.m;
+                const int kblocks = (K + BK - 1) / BK;
+                const uint32_t acc = local & 1;
+                const uint32_t acc_phase = (local >> 1) & 1;
+                if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.err, ERR_MMA_ACC)) { ok = false; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait(&full[stage], phase, abort_flag, p.err, ERR_MMA_SLOT)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(sA + stage * S2_A);
+                    const uint32_t b_base = smem_u32(sB + stage * S2_B);
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t adesc = smem_desc_sw128(a_base + kk * 32, 16, 1024);
+                        uint64_t bdesc;
+                        if (MODE == MODE_UPDATE) bdesc = smem_desc_sw128(b_base + kk * 2048, BK * 128, 1024);
+                        else bdesc = smem_desc_sw128(b_base + kk * 32, 16, 1024);
+                        tc_mma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    const uint32_t e_own = mapa_shared(smem_u32(&empty[stage]), 0);
+                    const uint32_t e_peer = mapa_shared(smem_u32(&empty[stage]), 1);
+                    tc_commit_pair(e_own);
+                    tc_commit_pair(e_peer);
+                    if (++stage == S2_STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) break;
+                tc_commit_pair(mapa_shared(smem_u32(&tfull[acc]), 0));
+                tc_commit_pair(mapa_shared(smem_u32(&tfull[acc]), 1));
+            }
+            if (!ok || *abort_flag) {
+                tc_commit_pair(mapa_shared(smem_u32(drain), 0));
+                const uint64_t t0 = globaltimer_ns();
+                while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 100000000ull) { }
+            }
+        }
+    } else {
+        const uint32_t q = warp & 3u;
+        const uint32_t half = (warp - 2) >> 2;
+        int local = 0;
+        for (int t = cid; t < p.ntiles; t += ncl, ++local) {
+            const int4 tile = p.tiles[t];
+            const GemmGroupInfo& gi = p.groups[tile.x];
+            const uint32_t acc = local & 1;
+            const uint32_t acc_phase = (local >> 1) & 1;
+            bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, ERR_EPILOGUE);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            tc_fence_after();
+            const int row = tile.z * S2_BM + (int)rank * 128 + (int)(q * 32 + lane);
+            epilogue_segment<MODE>(p, gi, tile.y, row, tile.w * S2_BN,
+                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * 128);
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync_all();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    }
+}
+
 }  // namespace
 
-size_t tc_gemm_smem_bytes() { return SMEM_BYTES; }
+size_t tc_gemm_smem_bytes(int pair) { return pair ? S2_SMEM : S1_SMEM; }
 int tc_gemm_threads() { return NUM_THREADS; }
+int tc_gemm_tile_m(int pair) { return pair ? S2_BM : S1_BM; }
+int tc_gemm_tile_n(int pair) { return pair ? S2_BN : S1_BN; }
 
 cudaError_t tc_gemm_prepare() {
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(ns_gemm_tc_kernel<MODE_GRAM>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(ns_gemm_tc_kernel<MODE_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES)) != cudaSuccess) return e;
-    return cudaFuncSetAttribute(ns_gemm_tc_kernel<MODE_UPDATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc_kernel<MODE_GRAM>, cudaFuncAttributeMaxDynamicSharedMemorySize, S1_SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc_kernel<MODE_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, S1_SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc_kernel<MODE_UPDATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, S1_SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_GRAM>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM)) != cudaSuccess) return e;
+    return cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_UPDATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM);
 }
 
-cudaError_t launch_tc_gemm(int mode, const GemmParams& p, int grid, cudaStream_t s) {
+cudaError_t tc_gemm_max_clusters(int* n) {
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3(2, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.dynamicSmemBytes = S2_SMEM;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaOccupancyMaxActiveClusters(n, ns_gemm_tc2_kernel<MODE_UPDATE>, &cfg);
+}
+
+cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cudaStream_t s) {
     if (p.ntiles <= 0) return cudaSuccess;
-    switch (mode) {
-        case MODE_GRAM: ns_gemm_tc_kernel<MODE_GRAM><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(p); break;
-        case MODE_POLY: ns_gemm_tc_kernel<MODE_POLY><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(p); break;
-        default: ns_gemm_tc_kernel<MODE_UPDATE><<<grid, NUM_THREADS, SMEM_BYTES, s>>>(p); break;
+    if (pair) {
+        switch (mode) {
+            case MODE_GRAM: ns_gemm_tc2_kernel<MODE_GRAM><<<grid, NUM_THREADS, S2_SMEM, s>>>(p); break;
+            case MODE_POLY: ns_gemm_tc2_kernel<MODE_POLY><<<grid, NUM_THREADS, S2_SMEM, s>>>(p); break;
+            default: ns_gemm_tc2_kernel<MODE_UPDATE><<<grid, NUM_THREADS, S2_SMEM, s>>>(p); break;
+        }
+    } else {
+        switch (mode) {
+            case MODE_GRAM: ns_gemm_tc_kernel<MODE_GRAM><<<grid, NUM_THREADS, S1_SMEM, s>>>(p); break;
+            case MODE_POLY: ns_gemm_tc_kernel<MODE_POLY><<<grid, NUM_THREADS, S1_SMEM, s>>>(p); break;
+            default: ns_gemm_tc_kernel<MODE_UPDATE><<<grid, NUM_THREADS, S1_SMEM, s>>>(p); break;
+        }
     }
     return cudaGetLastError();
 }

@@ -78,10 +78,19 @@ struct GemmParams {
     int* err;                     // device error word (bounded waits)
 };
 
-size_t tc_gemm_smem_bytes();
+// pair = 1: the two-CTA kernel (256 x 256 tiles, grid = 2 x clusters);
+// pair = 0: the one-CTA kernel (128 x 256 tiles).
+size_t tc_gemm_smem_bytes(int pair);
 int tc_gemm_threads();
+int tc_gemm_tile_m(int pair);
+int tc_gemm_tile_n(int pair);
 cudaError_t tc_gemm_prepare();    // sets the dynamic shared-memory attribute once per device
-cudaError_t launch_tc_gemm(int mode, const GemmParams& p, int grid, cudaStream_t s);
+cudaError_t tc_gemm_max_clusters(int* n);
+cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cudaStream_t s);
+
+// Default GEMM variant of new handles and planner queries: the two-CTA kernel unless
+// the environment variable MUON_GEMM_PAIR is "0".
+int tc_gemm_default_pair();
 
 // fp32 FFMA debug GEMM: C = alpha_eff * A op(B) + beta_eff * Cin, batched over `count`.
 // op(B)[k][j] = B[j][k] when b_kmajor, else B[k][j].  With `scale`, alpha_eff =

@@ -2,6 +2,8 @@
 #include "plan.h"
 
 #include <algorithm>
+#include <cstdlib>
+#include <cstring>
 
 namespace muon {
 
@@ -48,6 +50,11 @@ std::vector<Tile> build_tiles(const std::vector<GroupDims>& groups, int phase, i
     out.reserve(tiles.size());
     for (int i : order) out.push_back(tiles[i]);
     return out;
+}
+
+int tc_gemm_default_pair() {
+    const char* v = std::getenv("MUON_GEMM_PAIR");
+    return (v && std::strcmp(v, "0") == 0) ? 0 : 1;
 }
 
 }  // namespace muon

@@ -26,4 +26,7 @@ GroupDims make_dims(int rows, int cols, int count);
 // descending, ties in (group, matrix, tile_row, tile_col) order.
 std::vector<Tile> build_tiles(const std::vector<GroupDims>& groups, int phase, int bm, int bn);
 
+// 1 unless the environment variable MUON_GEMM_PAIR is "0" (see kernels.cuh).
+int tc_gemm_default_pair();
+
 }  // namespace muon

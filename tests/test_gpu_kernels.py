@@ -2,6 +2,8 @@
 path and fp32 debug path) through muon_ns_phase_run, each against the oracle's
 piece of eq. 4 (gram, poly_matrix, ns_update) on the same bf16 inputs widened
 exactly to fp64.  Sizes span several 128x256 tiles with ragged tails."""
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -13,10 +15,19 @@ from muon_newton_schulz_04_b200 import build as mbuild
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module")
-def opt():
+@pytest.fixture(scope="module", params=["pair", "single"])
+def opt(request):
+    """A handle on the two-CTA GEMM kernel (default) and one on the one-CTA kernel."""
     mbuild.build()
-    o = mb.Muon(mb.config())
+    old = os.environ.get("MUON_GEMM_PAIR")
+    os.environ["MUON_GEMM_PAIR"] = "1" if request.param == "pair" else "0"
+    try:
+        o = mb.Muon(mb.config())
+    finally:
+        if old is None:
+            del os.environ["MUON_GEMM_PAIR"]
+        else:
+            os.environ["MUON_GEMM_PAIR"] = old
     yield o
     o.close()
 
@@ -29,7 +40,7 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
-SHAPES = [(128, 256, 1), (320, 776, 3), (384, 384, 2), (136, 1032, 1), (8, 64, 2), (520, 264, 1)]
+SHAPES = [(128, 256, 1), (320, 776, 3), (384, 384, 2), (136, 1032, 1), (8, 64, 2), (520, 264, 1), (1024, 1536, 1)]
 
 
 @pytest.mark.parametrize("m,n,count", SHAPES)
