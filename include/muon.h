@@ -240,6 +240,15 @@ int muon_plan_tile_m(void);
 int muon_plan_tile_n(void);
 muon_status muon_plan_tiles(const int* shapes, int n_groups, int phase, int* out, int cap, int* n_tiles);
 
+/* Work units of one launch of the two-CTA GEMM kernel built for `clusters`
+ * two-CTA clusters: 10 ints per unit (cluster, group, matrix, tile_row, tile_col,
+ * k_begin, k_end, kind, slot, nslots), k in 64-element blocks.  kind 0 = a whole
+ * tile; 1 = the first K range of a split tile, which adds the partial sums of
+ * slots [slot, slot + nslots); 2 = a later K range, which stores its partial sum
+ * to `slot`.  Same conventions as muon_plan_tiles. */
+muon_status muon_plan_units(const int* shapes, int n_groups, int phase, int clusters, int* out, int cap,
+                            int* n_units);
+
 #ifdef __cplusplus
 }
 #endif

@@ -25,6 +25,8 @@ SOURCES = ["api.cu", "elementwise.cu", "gemm_tc.cu", "gemm_simt.cu", "plan.cpp",
 HEADERS = ["kernels.cuh", "ptx.cuh", "plan.h"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+# extra nvcc flags for experiments with compile-time constants (e.g. -DMUON_S2_STAGES=7)
+EXTRA = os.environ.get("MUON_NVCC_EXTRA", "").split()
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O3", "-Xptxas", "-v",
               "--expt-relaxed-constexpr", f"-I{os.path.join(ROOT, 'include')}"]
 
@@ -52,7 +54,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
         op = os.path.join(BUILD, src + ".o")
         objs.append(op)
         if force or not os.path.exists(op) or os.path.getmtime(op) < max(os.path.getmtime(sp), dep_t):
-            jobs.append([nvcc, *ARCH, *NVCC_FLAGS, "-x", "cu" if src.endswith(".cu") else "c++", "-c", sp, "-o", op])
+            jobs.append([nvcc, *ARCH, *NVCC_FLAGS, *EXTRA, "-x", "cu" if src.endswith(".cu") else "c++", "-c", sp, "-o", op])
 
     def run(cmd):
         r = subprocess.run(cmd, capture_output=True, text=True)

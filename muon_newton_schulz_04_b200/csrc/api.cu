@@ -3,7 +3,8 @@
 // Muon step ("Muon: An optimizer for hidden layers in neural networks",
 // section 4):
 //
-//   momentum_norm  ->  norm_finalize  ->  ns_steps x (GRAM -> POLY -> UPDATE)  ->  apply
+//   momentum_norm  ->  ns_steps x (GRAM -> POLY -> UPDATE)
+//   (the last UPDATE applies W; the fp32 debug path and ns_steps = 0 use the apply kernel)
 //
 // All launches go to the caller's stream; nothing here synchronises except the
 // entry points documented to do so.
@@ -11,6 +12,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 #include <string>
 #include <vector>
 
@@ -50,12 +52,20 @@ struct Plan {
     int n_gram = 0, n_poly = 0, n_upd = 0;
     // device addresses inside the workspace
     int4* d_tiles_gram = nullptr; int4* d_tiles_poly = nullptr; int4* d_tiles_upd = nullptr;
+    // two-CTA kernel: per-phase unit lists (plan.h) and the split-tile partial sums
+    int4* d_units[3] = {nullptr, nullptr, nullptr};
+    int* d_unit_begin[3] = {nullptr, nullptr, nullptr};
+    int unit_clusters = 0;
+    float* d_sk_partial = nullptr;
+    int* d_sk_count = nullptr;
+    int* d_sk_flag = nullptr;
     GemmMaps* d_maps = nullptr;
     GemmGroupInfo* d_ginfo = nullptr;
     EwSeg* d_segs = nullptr;
     double* d_partials = nullptr;
     float* d_norms = nullptr;
     float* d_scale = nullptr;
+    int* d_counters = nullptr;           // per-matrix block counters of the momentum kernel
     bool valid = false;
     std::vector<EwSeg> uploaded;         // last segment table copied to the device
 };
@@ -75,6 +85,7 @@ struct muon_handle {
     int* d_err = nullptr;
     Plan plan;
     EncodeTiledFn encode = nullptr;
+    int epoch = 0;           // distinct per two-CTA GEMM launch (split-tile flags)
     bool tc_ready = false;
     // per-phase timing
     bool timing = false;
@@ -83,6 +94,9 @@ struct muon_handle {
     std::vector<Pending> pending;
     double t_ms[MUON_TIMING_KINDS] = {};
     int t_n[MUON_TIMING_KINDS] = {};
+    // muon_step_host: side stream for copies that overlap the GEMMs, and its events
+    cudaStream_t side = nullptr;
+    cudaEvent_t ev_start = nullptr, ev_w = nullptr, ev_k1 = nullptr, ev_done = nullptr;
 };
 
 namespace {
@@ -251,8 +265,9 @@ muon_status encode_map(muon_handle* h, CUtensorMap* m, const void* base, int col
 bool is_bf16_path(const muon_handle* h) { return h->cfg.precision == MUON_PREC_BF16; }
 
 // Persistent grid: one CTA (or one two-CTA cluster) per tile, at most one per SM.
+// The two-CTA kernel runs one pair per unit list (lists are built for max_clusters).
 int gemm_grid(const muon_handle* h, int ntiles) {
-    if (h->pair) return 2 * std::min(ntiles, h->max_clusters);
+    if (h->pair) return 2 * h->max_clusters;
     return std::min(ntiles, h->num_sms);
 }
 
@@ -302,11 +317,32 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
     P.k1_blocks = k1;
     P.k7_blocks = k7;
     std::vector<Tile> tg, tp, tu;
+    UnitPlan upl[3];
+    int sk_slots = 0;
     if (bf16) {
+        if (!h->tc_ready) {
+            CUDA_TRY(h, tc_gemm_prepare());
+            CUDA_TRY(h, tc_gemm_max_clusters(&h->max_clusters));
+            if (h->max_clusters < 1) return fail(h, MUON_ERR_UNSUPPORTED, "no two-CTA cluster fits on this device");
+            h->tc_ready = true;
+        }
         const int bm = tc_gemm_tile_m(h->pair), bn = tc_gemm_tile_n(h->pair);
         tg = build_tiles(P.dims, 0, bm, bn);
         tp = build_tiles(P.dims, 1, bm, bn);
         tu = build_tiles(P.dims, 2, bm, bn);
+        if (h->pair) {
+            const std::vector<Tile>* lists[3] = {&tg, &tp, &tu};
+            for (int ph = 0; ph < 3; ++ph) {
+                std::vector<int> kb;
+                for (const Tile& t : *lists[ph]) {
+                    const GroupDims& d = P.dims[t.group];
+                    kb.push_back(((ph == 0 ? d.n : d.m) + TC_BK - 1) / TC_BK);
+                }
+                upl[ph] = build_units(*lists[ph], kb, h->max_clusters, tc_gemm_split_tiles() != 0);
+                sk_slots = std::max(sk_slots, upl[ph].nslots);
+            }
+            P.unit_clusters = h->max_clusters;
+        }
     }
     P.n_gram = (int)tg.size(); P.n_poly = (int)tp.size(); P.n_upd = (int)tu.size();
     const size_t o_tg = take(tg.size() * sizeof(int4) + 16), o_tp = take(tp.size() * sizeof(int4) + 16),
@@ -314,18 +350,39 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
     const size_t o_maps = take(ng * sizeof(GemmMaps)), o_ginfo = take(ng * sizeof(GemmGroupInfo));
     const size_t o_segs = take(P.segs.size() * sizeof(EwSeg)), o_part = take((size_t)k1 * sizeof(double) + 8);
     const size_t o_norm = take((size_t)mat * sizeof(float)), o_scale = take((size_t)mat * sizeof(float));
+    const size_t o_cnt = take((size_t)mat * sizeof(int));
+    size_t o_units[3], o_ubeg[3];
+    for (int ph = 0; ph < 3; ++ph) {
+        o_units[ph] = take(upl[ph].units.size() * 2 * sizeof(int4) + 32);
+        o_ubeg[ph] = take(upl[ph].begin.size() * sizeof(int) + 16);
+    }
+    const size_t o_skp = take((size_t)sk_slots * SK_SLOT_FLOATS * sizeof(float) + 16);
+    const size_t o_skc = take((size_t)sk_slots * sizeof(int) + 16), o_skf = take((size_t)sk_slots * sizeof(int) + 16);
     muon_status st = ensure_buf(h, h->ws, off);
     if (st != MUON_OK) { P.valid = false; return st; }
     char* base = static_cast<char*>(h->ws.ptr);
     P.d_tiles_gram = reinterpret_cast<int4*>(base + o_tg);
     P.d_tiles_poly = reinterpret_cast<int4*>(base + o_tp);
     P.d_tiles_upd = reinterpret_cast<int4*>(base + o_tu);
+    for (int ph = 0; ph < 3; ++ph) {
+        P.d_units[ph] = reinterpret_cast<int4*>(base + o_units[ph]);
+        P.d_unit_begin[ph] = reinterpret_cast<int*>(base + o_ubeg[ph]);
+    }
+    P.d_sk_partial = reinterpret_cast<float*>(base + o_skp);
+    P.d_sk_count = reinterpret_cast<int*>(base + o_skc);
+    P.d_sk_flag = reinterpret_cast<int*>(base + o_skf);
+    if (sk_slots > 0) {
+        CUDA_TRY(h, cudaMemsetAsync(P.d_sk_count, 0, (size_t)sk_slots * sizeof(int), s));
+        CUDA_TRY(h, cudaMemsetAsync(P.d_sk_flag, 0, (size_t)sk_slots * sizeof(int), s));
+    }
     P.d_maps = reinterpret_cast<GemmMaps*>(base + o_maps);
     P.d_ginfo = reinterpret_cast<GemmGroupInfo*>(base + o_ginfo);
     P.d_segs = reinterpret_cast<EwSeg*>(base + o_segs);
     P.d_partials = reinterpret_cast<double*>(base + o_part);
     P.d_norms = reinterpret_cast<float*>(base + o_norm);
     P.d_scale = reinterpret_cast<float*>(base + o_scale);
+    P.d_counters = reinterpret_cast<int*>(base + o_cnt);
+    CUDA_TRY(h, cudaMemsetAsync(P.d_counters, 0, (size_t)mat * sizeof(int), s));
 
     // workspace pointers in the segment table
     int mi = 0;
@@ -369,16 +426,22 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
         CUDA_TRY(h, up_tiles(P.d_tiles_gram, tg));
         CUDA_TRY(h, up_tiles(P.d_tiles_poly, tp));
         CUDA_TRY(h, up_tiles(P.d_tiles_upd, tu));
+        std::vector<std::vector<int4>> uv(3);
+        for (int ph = 0; ph < 3 && h->pair; ++ph) {
+            for (const Unit& u : upl[ph].units) {
+                uv[ph].push_back(make_int4(u.tile.group, u.tile.mat, u.tile.tile_row, u.tile.tile_col));
+                uv[ph].push_back(make_int4(u.k_begin, u.k_end, u.kind, u.slot | (u.nslots << 16)));
+            }
+            if (!uv[ph].empty())
+                CUDA_TRY(h, cudaMemcpyAsync(P.d_units[ph], uv[ph].data(), uv[ph].size() * sizeof(int4),
+                                            cudaMemcpyHostToDevice, s));
+            CUDA_TRY(h, cudaMemcpyAsync(P.d_unit_begin[ph], upl[ph].begin.data(), upl[ph].begin.size() * sizeof(int),
+                                        cudaMemcpyHostToDevice, s));
+        }
         CUDA_TRY(h, cudaMemcpyAsync(P.d_maps, maps.data(), ng * sizeof(GemmMaps), cudaMemcpyHostToDevice, s));
         CUDA_TRY(h, cudaMemcpyAsync(P.d_ginfo, gi.data(), ng * sizeof(GemmGroupInfo), cudaMemcpyHostToDevice, s));
         // pageable copies are staged before return; wait so the host vectors may go
         CUDA_TRY(h, cudaStreamSynchronize(s));
-        if (!h->tc_ready) {
-            CUDA_TRY(h, tc_gemm_prepare());
-            CUDA_TRY(h, tc_gemm_max_clusters(&h->max_clusters));
-            if (h->max_clusters < 1) return fail(h, MUON_ERR_UNSUPPORTED, "no two-CTA cluster fits on this device");
-            h->tc_ready = true;
-        }
     }
     P.valid = true;
     return MUON_OK;
@@ -422,27 +485,48 @@ muon_status upload_segs(muon_handle* h, const std::vector<MatPtrs>& mp, cudaStre
     return MUON_OK;
 }
 
-muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStream_t s) {
+// Work that muon_step_host splices into the launch sequence.
+struct Hooks {
+    cudaEvent_t w_ready = nullptr;                    // s waits for it before W is first read
+    std::function<muon_status()> after_momentum;     // enqueued right after the momentum kernel
+};
+
+muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStream_t s, const Hooks* hooks = nullptr) {
     Plan& P = h->plan;
     const muon_config& c = h->cfg;
     const bool bf16 = is_bf16_path(h);
     TIMED(h, 0, s, launch_momentum_norm(P.d_segs, P.nmat, P.k1_blocks, P.d_partials, momentum ? c.momentum : 0.f,
-                                        momentum ? c.nesterov : 0, bf16 ? 1 : 0, s));
-    TIMED(h, 1, s, launch_norm_finalize(P.d_segs, P.nmat, P.d_partials, c.eps, P.d_norms, P.d_scale, s));
+                                        momentum ? c.nesterov : 0, bf16 ? 1 : 0, P.d_counters, c.eps, P.d_norms,
+                                        P.d_scale, s));
+    if (hooks && hooks->after_momentum) {
+        muon_status st = hooks->after_momentum();
+        if (st != MUON_OK) return st;
+    }
     char* base = static_cast<char*>(h->ws.ptr);
     for (int it = 0; it < c.ns_steps; ++it) {
         const int par = it & 1;
         if (bf16) {
             GemmParams gp{};
             gp.maps = P.d_maps; gp.groups = P.d_ginfo; gp.parity = par; gp.err = h->d_err;
+            gp.sk_partial = P.d_sk_partial; gp.sk_count = P.d_sk_count; gp.sk_flag = P.d_sk_flag;
             gp.tiles = P.d_tiles_gram; gp.ntiles = P.n_gram; gp.alpha = 1.f; gp.beta = 0.f;
+            gp.units = P.d_units[0]; gp.unit_begin = P.d_unit_begin[0]; gp.epoch = ++h->epoch;
             gp.scale = it == 0 ? P.d_scale : nullptr;
             TIMED(h, 2, s, launch_tc_gemm(MODE_GRAM, h->pair, gp, gemm_grid(h, P.n_gram), s));
             gp.tiles = P.d_tiles_poly; gp.ntiles = P.n_poly; gp.alpha = c.ns_c; gp.beta = c.ns_b; gp.scale = nullptr;
+            gp.units = P.d_units[1]; gp.unit_begin = P.d_unit_begin[1]; gp.epoch = ++h->epoch;
             TIMED(h, 3, s, launch_tc_gemm(MODE_POLY, h->pair, gp, gemm_grid(h, P.n_poly), s));
             gp.tiles = P.d_tiles_upd; gp.ntiles = P.n_upd; gp.alpha = 1.f; gp.beta = c.ns_a;
+            gp.units = P.d_units[2]; gp.unit_begin = P.d_unit_begin[2]; gp.epoch = ++h->epoch;
             gp.scale = it == 0 ? P.d_scale : nullptr;
             gp.write_op = (it + 1 < c.ns_steps) ? 1 : 0;
+            if (it + 1 == c.ns_steps) {        // fused apply / copy-out
+                if (hooks && hooks->w_ready) CUDA_TRY(h, cudaStreamWaitEvent(s, hooks->w_ready, 0));
+                gp.apply_mode = copy_out ? 2 : 1;
+                gp.decay = copy_out ? 1.f : 1.f - c.lr * c.weight_decay;
+                gp.lr = c.lr;
+                gp.segs = P.d_segs;
+            }
             TIMED(h, 4, s, launch_tc_gemm(MODE_UPDATE, h->pair, gp, gemm_grid(h, P.n_upd), s));
         } else {
             for (size_t g = 0; g < P.dims.size(); ++g) {
@@ -476,13 +560,16 @@ muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStrea
             }
         }
     }
+    if (bf16 && c.ns_steps > 0) return MUON_OK;
+    if (hooks && hooks->w_ready) CUDA_TRY(h, cudaStreamWaitEvent(s, hooks->w_ready, 0));
     const float decay = copy_out ? 1.f : 1.f - c.lr * c.weight_decay;
     TIMED(h, 5, s, launch_apply(P.d_segs, P.nmat, P.k7_blocks, decay, c.lr, c.ns_steps == 0 ? P.d_scale : nullptr,
                                 copy_out ? 1 : 0, s));
     return MUON_OK;
 }
 
-muon_status step_device(muon_handle* h, const muon_group* groups, int n, cudaStream_t s) {
+muon_status step_device(muon_handle* h, const muon_group* groups, int n, cudaStream_t s,
+                        const Hooks* hooks = nullptr) {
     std::vector<int> shapes;
     std::vector<MatPtrs> mp;
     for (int i = 0; i < n; ++i) {
@@ -494,7 +581,7 @@ muon_status step_device(muon_handle* h, const muon_group* groups, int n, cudaStr
     muon_status st = ensure_plan(h, shapes, s);
     if (st != MUON_OK) return st;
     if ((st = upload_segs(h, mp, s)) != MUON_OK) return st;
-    return run_pipeline(h, true, false, s);
+    return run_pipeline(h, true, false, s, hooks);
 }
 
 }  // namespace
@@ -600,6 +687,17 @@ muon_status muon_step_host(muon_handle* h, const muon_group* groups, int n_group
     std::vector<std::vector<float*>> Wd(n_groups), Bd(n_groups);
     std::vector<std::vector<const void*>> Gd(n_groups);
     std::vector<muon_group> dg_groups(groups, groups + n_groups);
+    if (!h->side) {
+        CUDA_TRY(h, cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
+        cudaEvent_t* evs[4] = {&h->ev_start, &h->ev_w, &h->ev_k1, &h->ev_done};
+        for (cudaEvent_t* e : evs) CUDA_TRY(h, cudaEventCreateWithFlags(e, cudaEventDisableTiming));
+    }
+    // The side stream starts after everything already queued on s (the staging
+    // area may still be in use by the previous call).  G and B go up on s; W goes
+    // up on the side stream and is waited for only before the weight update; B comes
+    // back on the side stream as soon as the momentum kernel has finished with it.
+    CUDA_TRY(h, cudaEventRecord(h->ev_start, s));
+    CUDA_TRY(h, cudaStreamWaitEvent(h->side, h->ev_start, 0));
     int mi = 0;
     for (int i = 0; i < n_groups; ++i) {
         const size_t e = (size_t)groups[i].rows * groups[i].cols;
@@ -609,21 +707,35 @@ muon_status muon_step_host(muon_handle* h, const muon_group* groups, int n_group
             float* b = reinterpret_cast<float*>(base + ob[mi]);
             void* g = base + og[mi];
             CUDA_TRY(h, cudaMemcpyAsync(g, groups[i].G[k], gsz, cudaMemcpyHostToDevice, s));
-            CUDA_TRY(h, cudaMemcpyAsync(w, groups[i].W[k], e * 4, cudaMemcpyHostToDevice, s));
             CUDA_TRY(h, cudaMemcpyAsync(b, groups[i].B[k], e * 4, cudaMemcpyHostToDevice, s));
+            CUDA_TRY(h, cudaMemcpyAsync(w, groups[i].W[k], e * 4, cudaMemcpyHostToDevice, h->side));
             Wd[i].push_back(w); Bd[i].push_back(b); Gd[i].push_back(g);
         }
         dg_groups[i].W = Wd[i].data(); dg_groups[i].B = Bd[i].data(); dg_groups[i].G = Gd[i].data();
     }
-    if ((st = step_device(h, dg_groups.data(), n_groups, s)) != MUON_OK) return st;
+    CUDA_TRY(h, cudaEventRecord(h->ev_w, h->side));
+    Hooks hooks;
+    hooks.w_ready = h->ev_w;
+    hooks.after_momentum = [&]() -> muon_status {
+        CUDA_TRY(h, cudaEventRecord(h->ev_k1, s));
+        CUDA_TRY(h, cudaStreamWaitEvent(h->side, h->ev_k1, 0));
+        int j = 0;
+        for (int i = 0; i < n_groups; ++i) {
+            const size_t e = (size_t)groups[i].rows * groups[i].cols;
+            for (int k = 0; k < groups[i].count; ++k, ++j)
+                CUDA_TRY(h, cudaMemcpyAsync(groups[i].B[k], base + ob[j], e * 4, cudaMemcpyDeviceToHost, h->side));
+        }
+        return MUON_OK;
+    };
+    if ((st = step_device(h, dg_groups.data(), n_groups, s, &hooks)) != MUON_OK) return st;
     mi = 0;
     for (int i = 0; i < n_groups; ++i) {
         const size_t e = (size_t)groups[i].rows * groups[i].cols;
-        for (int k = 0; k < groups[i].count; ++k, ++mi) {
+        for (int k = 0; k < groups[i].count; ++k, ++mi)
             CUDA_TRY(h, cudaMemcpyAsync(groups[i].W[k], base + ow[mi], e * 4, cudaMemcpyDeviceToHost, s));
-            CUDA_TRY(h, cudaMemcpyAsync(groups[i].B[k], base + ob[mi], e * 4, cudaMemcpyDeviceToHost, s));
-        }
     }
+    CUDA_TRY(h, cudaEventRecord(h->ev_done, h->side));
+    CUDA_TRY(h, cudaStreamWaitEvent(s, h->ev_done, 0));
     return MUON_OK;
 }
 
@@ -725,19 +837,48 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
         gi.xf_out = (float*)a->out;
         gi.xb[1] = (__nv_bfloat16*)a->out_op;
     }
-    const size_t o_maps = 0, o_gi = align_up(sizeof(GemmMaps), 256), o_t = o_gi + align_up(sizeof(GemmGroupInfo), 256);
-    const size_t need = o_t + tl.size() * sizeof(int4) + 16;
+    // unit lists of the two-CTA kernel (split tiles included, so the building
+    // blocks exercise the partial-sum path too)
+    UnitPlan up;
+    if (h->pair) {
+        std::vector<int> kb;
+        for (size_t i = 0; i < tl.size(); ++i) kb.push_back(((phase == MUON_NS_GRAM ? n : m) + TC_BK - 1) / TC_BK);
+        up = build_units(tl, kb, h->max_clusters, tc_gemm_split_tiles() != 0);
+    }
+    std::vector<int4> uv;
+    for (const Unit& u : up.units) {
+        uv.push_back(make_int4(u.tile.group, u.tile.mat, u.tile.tile_row, u.tile.tile_col));
+        uv.push_back(make_int4(u.k_begin, u.k_end, u.kind, u.slot | (u.nslots << 16)));
+    }
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = align_up(off, 256); off = o + align_up(bytes, 256); return o; };
+    const size_t o_maps = take(sizeof(GemmMaps)), o_gi = take(sizeof(GemmGroupInfo));
+    const size_t o_t = take(tl.size() * sizeof(int4) + 16), o_u = take(uv.size() * sizeof(int4) + 16);
+    const size_t o_ub = take(up.begin.size() * sizeof(int) + 16);
+    const size_t o_skp = take((size_t)up.nslots * SK_SLOT_FLOATS * sizeof(float) + 16);
+    const size_t o_skc = take((size_t)up.nslots * sizeof(int) + 16), o_skf = take((size_t)up.nslots * sizeof(int) + 16);
     // the scratch area may still be read by an earlier launch on another stream
     if (h->scratch.ptr) CUDA_TRY(h, cudaDeviceSynchronize());
-    if ((st = ensure_buf(h, h->scratch, need)) != MUON_OK) return st;
+    if ((st = ensure_buf(h, h->scratch, off)) != MUON_OK) return st;
     char* base = static_cast<char*>(h->scratch.ptr);
     std::vector<int4> tv(tl.size());
     for (size_t i = 0; i < tl.size(); ++i) tv[i] = make_int4(tl[i].group, tl[i].mat, tl[i].tile_row, tl[i].tile_col);
     CUDA_TRY(h, cudaMemcpyAsync(base + o_maps, &maps, sizeof(maps), cudaMemcpyHostToDevice, s));
     CUDA_TRY(h, cudaMemcpyAsync(base + o_gi, &gi, sizeof(gi), cudaMemcpyHostToDevice, s));
     CUDA_TRY(h, cudaMemcpyAsync(base + o_t, tv.data(), tv.size() * sizeof(int4), cudaMemcpyHostToDevice, s));
+    if (!uv.empty()) CUDA_TRY(h, cudaMemcpyAsync(base + o_u, uv.data(), uv.size() * sizeof(int4), cudaMemcpyHostToDevice, s));
+    if (!up.begin.empty())
+        CUDA_TRY(h, cudaMemcpyAsync(base + o_ub, up.begin.data(), up.begin.size() * sizeof(int), cudaMemcpyHostToDevice, s));
+    CUDA_TRY(h, cudaMemsetAsync(base + o_skc, 0, (size_t)up.nslots * sizeof(int) + 16, s));
+    CUDA_TRY(h, cudaMemsetAsync(base + o_skf, 0, (size_t)up.nslots * sizeof(int) + 16, s));
     CUDA_TRY(h, cudaStreamSynchronize(s));
     GemmParams gp{};
+    gp.units = reinterpret_cast<const int4*>(base + o_u);
+    gp.unit_begin = reinterpret_cast<const int*>(base + o_ub);
+    gp.sk_partial = reinterpret_cast<float*>(base + o_skp);
+    gp.sk_count = reinterpret_cast<int*>(base + o_skc);
+    gp.sk_flag = reinterpret_cast<int*>(base + o_skf);
+    gp.epoch = 1;
     gp.tiles = reinterpret_cast<const int4*>(base + o_t);
     gp.ntiles = (int)tl.size();
     gp.maps = reinterpret_cast<const GemmMaps*>(base + o_maps);
@@ -825,6 +966,9 @@ muon_status muon_destroy(muon_handle* h) {
         cudaDeviceSynchronize();
         for (auto& p : h->pending) { cudaEventDestroy(p.a); cudaEventDestroy(p.b); }
         for (auto e : h->ev_free) cudaEventDestroy(e);
+        cudaEvent_t evs[4] = {h->ev_start, h->ev_w, h->ev_k1, h->ev_done};
+        for (cudaEvent_t e : evs) if (e) cudaEventDestroy(e);
+        if (h->side) cudaStreamDestroy(h->side);
         if (h->ws.ptr) cudaFree(h->ws.ptr);
         if (h->staging.ptr) cudaFree(h->staging.ptr);
         if (h->scratch.ptr) cudaFree(h->scratch.ptr);
@@ -865,6 +1009,32 @@ muon_status muon_plan_tiles(const int* shapes, int n_groups, int phase, int* out
     if (!out || cap < (int)t.size()) return MUON_ERR_INVALID;
     for (size_t i = 0; i < t.size(); ++i) {
         out[4 * i] = t[i].group; out[4 * i + 1] = t[i].mat; out[4 * i + 2] = t[i].tile_row; out[4 * i + 3] = t[i].tile_col;
+    }
+    return MUON_OK;
+}
+
+muon_status muon_plan_units(const int* shapes, int n_groups, int phase, int clusters, int* out, int cap,
+                            int* n_units) {
+    if (!shapes || n_groups <= 0 || !n_units || phase < 0 || phase > 2 || clusters < 1) return MUON_ERR_INVALID;
+    std::vector<GroupDims> dims;
+    for (int g = 0; g < n_groups; ++g) {
+        std::string why;
+        if (check_shape(shapes[3 * g], shapes[3 * g + 1], shapes[3 * g + 2], &why) != MUON_OK) return MUON_ERR_INVALID;
+        dims.push_back(make_dims(shapes[3 * g], shapes[3 * g + 1], shapes[3 * g + 2]));
+    }
+    std::vector<Tile> t = build_tiles(dims, phase, tc_gemm_tile_m(1), tc_gemm_tile_n(1));
+    std::vector<int> kb;
+    for (const Tile& x : t) kb.push_back(((phase == 0 ? dims[x.group].n : dims[x.group].m) + TC_BK - 1) / TC_BK);
+    UnitPlan up = build_units(t, kb, clusters, true);
+    *n_units = (int)up.units.size();
+    if (!out || cap < (int)up.units.size()) return MUON_ERR_INVALID;
+    for (int c = 0; c < clusters; ++c) {
+        for (int i = up.begin[c]; i < up.begin[c + 1]; ++i) {
+            const Unit& u = up.units[i];
+            int* o = out + 10 * i;
+            o[0] = c; o[1] = u.tile.group; o[2] = u.tile.mat; o[3] = u.tile.tile_row; o[4] = u.tile.tile_col;
+            o[5] = u.k_begin; o[6] = u.k_end; o[7] = u.kind; o[8] = u.slot; o[9] = u.nslots;
+        }
     }
     return MUON_OK;
 }

@@ -5,7 +5,8 @@
 //                                                    and its Nesterov remark)
 //                  X0 <- U, or U^T when rows > cols  (section 4: smaller-Gram orientation)
 //                  per-block sum of U^2 in fp64      (section 4: Frobenius normalisation)
-//  norm_finalize   ||U||_F and s = 1/(||U||_F + eps) per matrix, summed in a fixed order
+//                  the last block of each matrix to finish sums that matrix's
+//                  partials in a fixed order: ||U||_F and s = 1/(||U||_F + eps)
 //  apply           W <- (1 - lr*wd) W - lr*s_shape*O (eq. 3 with decoupled decay and the
 //                  per-shape scale of the Moonlight result), O read back transposed
 //                  when the matrix was oriented; or O copied out (orthogonalisation only)
@@ -57,7 +58,9 @@ __device__ __forceinline__ float direction(float g, float* bptr, float mu, int n
 
 __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* __restrict__ segs, int nseg,
                                                                   double* __restrict__ partials, float mu,
-                                                                  int nesterov, int bf16_operand) {
+                                                                  int nesterov, int bf16_operand,
+                                                                  int* __restrict__ counters, float eps,
+                                                                  float* __restrict__ norms, float* __restrict__ scale) {
     __shared__ float tile[EW_TILE][EW_TILE + 1];
     __shared__ double red[EW_THREADS / 32];
     const int si = find_seg(segs, nseg, blockIdx.x, false);
@@ -150,24 +153,28 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* 
         }
     }
     const double tot = block_sum(acc, red);
-    if (threadIdx.x == 0) partials[blockIdx.x] = tot;
-}
-
-// One warp per matrix: fixed-order sum of its block partials.
-__global__ void norm_finalize_kernel(const EwSeg* __restrict__ segs, int nseg, const double* __restrict__ partials,
-                                     float eps, float* __restrict__ norms, float* __restrict__ scale) {
-    const int wid = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (wid >= nseg) return;
-    const EwSeg& sg = segs[wid];
-    double s = 0.0;
-    for (int i = lane; i < sg.blk_count; i += 32) s += partials[sg.blk_begin + i];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) s += __shfl_down_sync(0xffffffffu, s, o);
-    if (lane == 0) {
-        const double nrm = sqrt(s);
+    __shared__ int is_last;
+    if (threadIdx.x == 0) {
+        partials[blockIdx.x] = tot;
+        __threadfence();
+        is_last = atomicAdd(&counters[sg.mat], 1) == sg.blk_count - 1;
+    }
+    __syncthreads();
+    if (!is_last) return;
+    // Last block of this matrix: every partial is visible.  Thread t sums partials
+    // t, t + 256, ...; the block reduction then adds them in a fixed order, so the
+    // result does not depend on which block finished last.
+    __threadfence();
+    double s2 = 0.0;
+    for (int i = threadIdx.x; i < sg.blk_count; i += EW_THREADS)
+        s2 += reinterpret_cast<volatile double*>(partials)[sg.blk_begin + i];
+    __syncthreads();
+    const double total = block_sum(s2, red);
+    if (threadIdx.x == 0) {
+        const double nrm = sqrt(total);
         norms[sg.mat] = (float)nrm;
         scale[sg.mat] = (float)(1.0 / (nrm + (double)eps));
+        counters[sg.mat] = 0;           // ready for the next call
     }
 }
 
@@ -242,18 +249,11 @@ __global__ void __launch_bounds__(EW_THREADS) copy_out_one_kernel(const EwSeg sg
 }  // namespace
 
 cudaError_t launch_momentum_norm(const EwSeg* segs, int nseg, int nblocks, double* partials, float mu,
-                                 int nesterov, int bf16_operand, cudaStream_t s) {
-    if (nblocks <= 0) return cudaSuccess;
-    momentum_norm_kernel<<<nblocks, EW_THREADS, 0, s>>>(segs, nseg, partials, mu, nesterov, bf16_operand);
-    return cudaGetLastError();
-}
-
-cudaError_t launch_norm_finalize(const EwSeg* segs, int nseg, const double* partials, float eps, float* norms,
+                                 int nesterov, int bf16_operand, int* counters, float eps, float* norms,
                                  float* scale, cudaStream_t s) {
-    if (nseg <= 0) return cudaSuccess;
-    const int threads = 256;
-    const int blocks = (nseg * 32 + threads - 1) / threads;
-    norm_finalize_kernel<<<blocks, threads, 0, s>>>(segs, nseg, partials, eps, norms, scale);
+    if (nblocks <= 0) return cudaSuccess;
+    momentum_norm_kernel<<<nblocks, EW_THREADS, 0, s>>>(segs, nseg, partials, mu, nesterov, bf16_operand, counters,
+                                                        eps, norms, scale);
     return cudaGetLastError();
 }
 

@@ -51,14 +51,43 @@ constexpr int S1_B = S1_BN * BK * 2;          // 32 KiB
 constexpr int S1_SMEM = 1024 + S1_STAGES * (S1_A + S1_B) + 256;
 
 // two-CTA kernel (per CTA)
-constexpr int S2_BM = 256, S2_BN = 256, S2_STAGES = 6;
+#ifndef MUON_S2_STAGES
+#define MUON_S2_STAGES 6
+#endif
+constexpr int S2_BM = 256, S2_BN = 256, S2_STAGES = MUON_S2_STAGES;
 constexpr int S2_A = 128 * BK * 2;            // 16 KiB: this CTA's 128 rows of A
 constexpr int S2_B = 128 * BK * 2;            // 16 KiB: this CTA's 128 columns of B
 constexpr int S2_SMEM = 1024 + S2_STAGES * (S2_A + S2_B) + 256;
 
 // error codes written to the device error word when a bounded wait gives up
 constexpr int ERR_PRODUCER = 0x101, ERR_MMA_SLOT = 0x102, ERR_MMA_ACC = 0x103, ERR_EPILOGUE = 0x104,
-              ERR_TAIL = 0x105;
+              ERR_TAIL = 0x105, ERR_SPLIT = 0x106;
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_gpu(int* p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" :: "l"(p), "r"(v) : "memory");
+}
+
+// Bounded wait until *flag == value (a partial sum published by another cluster).
+__device__ __forceinline__ bool flag_wait(const int* flag, int value, volatile int* abort_flag, int* err, int code) {
+    if (ld_acquire_gpu(flag) == value) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        __nanosleep(64);
+        if (ld_acquire_gpu(flag) == value) return true;
+        if (*abort_flag) return false;
+        if (globaltimer_ns() - t0 > MUON_WAIT_NS) {
+            atomicCAS(err, 0, code);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -101,13 +130,65 @@ __device__ __forceinline__ void store_symmetric(__nv_bfloat16* __restrict__ out,
     }
 }
 
+// Update of the weight (apply_mode 1: W <- decay*W - lr*s*O, eq. 3 with decoupled
+// decay and the per-shape scale) or copy-out of O (apply_mode 2) for the 32
+// finished values O[row][col0..col0+31] of the oriented result.  A matrix that was
+// transposed for the smaller Gram gets W[c][row]: lanes hold consecutive rows, so
+// each store instruction of the warp covers 32 consecutive elements of W's row c.
+__device__ __forceinline__ void apply_chunk(const GemmParams& p, const GemmGroupInfo& gi, int mat, int row,
+                                            int col0, const float (&val)[32]) {
+    const EwSeg& sg = p.segs[gi.mat_base + mat];
+    float* w = sg.w;
+    const float step = p.lr * sg.update_scale;
+    const bool copy = p.apply_mode == 2;
+    if (!sg.transposed) {
+        float* wr = w + (size_t)row * sg.cols;
+        if (sg.vec && col0 + 31 < gi.n) {
+            float4* w4 = reinterpret_cast<float4*>(wr + col0);
+#pragma unroll
+            for (int qq = 0; qq < 8; ++qq) {
+                float4 o = make_float4(val[4 * qq], val[4 * qq + 1], val[4 * qq + 2], val[4 * qq + 3]);
+                if (!copy) {
+                    const float4 x = w4[qq];
+                    o.x = fmaf(-step, o.x, p.decay * x.x);
+                    o.y = fmaf(-step, o.y, p.decay * x.y);
+                    o.z = fmaf(-step, o.z, p.decay * x.z);
+                    o.w = fmaf(-step, o.w, p.decay * x.w);
+                }
+                w4[qq] = o;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int c = col0 + j;
+                if (c < gi.n) wr[c] = copy ? val[j] : fmaf(-step, val[j], p.decay * wr[c]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int c = col0 + j;
+            if (c < gi.n) {
+                float* wp = w + (size_t)c * sg.cols + row;
+                *wp = copy ? val[j] : fmaf(-step, val[j], p.decay * *wp);
+            }
+        }
+    }
+}
+
 // Epilogue of one accumulator row segment: 4 chunks of 32 columns starting at
 // column `c_begin` of the accumulator whose TMEM address (lane quarter included)
 // is `tacc`.  `row` is the global output row of this thread, `col_base` the
 // global column of accumulator column 0.
+//
+// Split tiles (two-CTA kernel): kind 2 stores the raw fp32 accumulator row to its
+// partial-sum slot at `sk_row` and does nothing else; kind 1 adds the `nslots`
+// partial rows at sk_row, sk_row + SK_SLOT_FLOATS, ... (in K order) before the
+// usual epilogue; kind 0 is a whole tile.
 template <int MODE>
 __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const GemmGroupInfo& gi, int mat, int row,
-                                                 int col_base, uint32_t tacc, int c_begin) {
+                                                 int col_base, uint32_t tacc, int c_begin, int kind = 0,
+                                                 float* sk_row = nullptr, int nslots = 0) {
     float alpha = p.alpha, beta = p.beta;
     if (p.scale != nullptr) {
         const float s = p.scale[gi.mat_base + mat];
@@ -120,6 +201,27 @@ __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const Gemm
         uint32_t v[32];
         tmem_ld_32x32b_x32(tacc + (uint32_t)c_local, v);
         tmem_ld_wait();
+        if (kind == 2) {
+            float4* dst = reinterpret_cast<float4*>(sk_row + c_local);
+#pragma unroll
+            for (int qq = 0; qq < 8; ++qq)
+                dst[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
+                                      __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
+            continue;
+        }
+        if (kind == 1) {
+            for (int sl = 0; sl < nslots; ++sl) {
+                const float4* src = reinterpret_cast<const float4*>(sk_row + (size_t)sl * SK_SLOT_FLOATS + c_local);
+#pragma unroll
+                for (int qq = 0; qq < 8; ++qq) {
+                    const float4 x = __ldcg(src + qq);
+                    v[4 * qq + 0] = __float_as_uint(__uint_as_float(v[4 * qq + 0]) + x.x);
+                    v[4 * qq + 1] = __float_as_uint(__uint_as_float(v[4 * qq + 1]) + x.y);
+                    v[4 * qq + 2] = __float_as_uint(__uint_as_float(v[4 * qq + 2]) + x.z);
+                    v[4 * qq + 3] = __float_as_uint(__uint_as_float(v[4 * qq + 3]) + x.w);
+                }
+            }
+        }
         const int col0 = col_base + c_local;
         float val[32];
         if (MODE == MODE_GRAM) {
@@ -185,13 +287,15 @@ __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const Gemm
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int c = col0 + j;
+                        const float r = (c < gi.n) ? alpha * __uint_as_float(v[j]) + beta * xin[c] : 0.f;
+                        val[j] = r;
                         if (c < gi.n) {
-                            const float r = alpha * __uint_as_float(v[j]) + beta * xin[c];
                             xout[c] = r;
                             if (p.write_op) xb[c] = __float2bfloat16_rn(r);
                         }
                     }
                 }
+                if (p.apply_mode != 0) apply_chunk(p, gi, mat, row, col0, val);
             }
         }
     }
@@ -387,8 +491,7 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
     const uint32_t warp = warp_id();
     const uint32_t lane = threadIdx.x & 31u;
     const uint32_t rank = cluster_ctarank();          // 0: issues the MMA
-    const int cid = (int)cluster_id_x();
-    const int ncl = (int)nclusters_x();
+    const int cid = (int)cluster_id_x();               // index of this pair's unit list
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < S2_STAGES; ++s) {
@@ -416,17 +519,16 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
         if (elect_one()) {
             uint32_t stage = 0, phase = 0;
             bool ok = true;
-            for (int t = cid; t < p.ntiles && ok; t += ncl) {
-                const int4 tile = p.tiles[t];
-                const GemmGroupInfo& gi = p.groups[tile.x];
-                const int K = (MODE == MODE_GRAM) ? gi.n : gi.m;
-                const int kblocks = (K + BK - 1) / BK;
+            const int u_end = p.unit_begin[cid + 1];
+            for (int u = p.unit_begin[cid]; u < u_end && ok; ++u) {
+                const int4 tile = p.units[2 * u];
+                const int4 sk = p.units[2 * u + 1];
                 const void *mapA, *mapB;
                 operand_maps<MODE>(p, tile.x, mapA, mapB);
                 const int row0 = tile.z * S2_BM + (int)rank * 128;     // this CTA's rows of A
                 const int colh = tile.w * S2_BN + (int)rank * 128;     // this CTA's columns of B
                 const int mat = tile.y;
-                for (int kb = 0; kb < kblocks; ++kb) {
+                for (int kb = sk.x; kb < sk.y; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, ERR_PRODUCER)) { ok = false; break; }
                     const uint32_t full0 = mapa_shared(smem_u32(&full[stage]), 0);
                     if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2 * (S2_A + S2_B));
@@ -455,17 +557,15 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
             uint32_t stage = 0, phase = 0;
             int local = 0;
             bool ok = true;
-            for (int t = cid; t < p.ntiles && ok; t += ncl, ++local) {
-                const int4 tile = p.tiles[t];
-                const GemmGroupInfo& gi = p.groups[tile.x];
-                const int K = (MODE == MODE_GRAM) ? gi.n : gi.m;
-                const int kblocks = (K + BK - 1) / BK;
+            const int u_end = p.unit_begin[cid + 1];
+            for (int u = p.unit_begin[cid]; u < u_end && ok; ++u, ++local) {
+                const int4 sk = p.units[2 * u + 1];
                 const uint32_t acc = local & 1;
                 const uint32_t acc_phase = (local >> 1) & 1;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.err, ERR_MMA_ACC)) { ok = false; break; }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + acc * ACC_COLS;
-                for (int kb = 0; kb < kblocks; ++kb) {
+                for (int kb = sk.x; kb < sk.y; ++kb) {
                     if (!mbar_wait(&full[stage], phase, abort_flag, p.err, ERR_MMA_SLOT)) { ok = false; break; }
                     tc_fence_after();
                     const uint32_t a_base = smem_u32(sA + stage * S2_A);
@@ -476,7 +576,7 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
                         uint64_t bdesc;
                         if (MODE == MODE_UPDATE) bdesc = smem_desc_sw128(b_base + kk * 2048, BK * 128, 1024);
                         else bdesc = smem_desc_sw128(b_base + kk * 32, 16, 1024);
-                        tc_mma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb | kk) != 0 ? 1u : 0u);
+                        tc_mma_f16_pair(d_tmem, adesc, bdesc, idesc, (kb != sk.x || kk != 0) ? 1u : 0u);
                     }
                     const uint32_t e_own = mapa_shared(smem_u32(&empty[stage]), 0);
                     const uint32_t e_peer = mapa_shared(smem_u32(&empty[stage]), 1);
@@ -498,20 +598,42 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
         const uint32_t q = warp & 3u;
         const uint32_t half = (warp - 2) >> 2;
         int local = 0;
-        for (int t = cid; t < p.ntiles; t += ncl, ++local) {
-            const int4 tile = p.tiles[t];
+        const int u_end = p.unit_begin[cid + 1];
+        for (int u = p.unit_begin[cid]; u < u_end; ++u, ++local) {
+            const int4 tile = p.units[2 * u];
+            const int4 sk = p.units[2 * u + 1];
+            const int kind = sk.z, slot = sk.w & 0xFFFF, nsl = sk.w >> 16;
             const GemmGroupInfo& gi = p.groups[tile.x];
             const uint32_t acc = local & 1;
             const uint32_t acc_phase = (local >> 1) & 1;
             bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, ERR_EPILOGUE);
+            if (kind == 1 && lane == 0) {
+                // the later parts of this split tile, produced first by other clusters
+                for (int sl = 0; sl < nsl && ok; ++sl)
+                    ok = flag_wait(&p.sk_flag[slot + sl], p.epoch, abort_flag, p.err, ERR_SPLIT);
+            }
+            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const int row = tile.z * S2_BM + (int)rank * 128 + (int)(q * 32 + lane);
+            const int row_local = (int)(q * 32 + lane);
+            const int row = tile.z * S2_BM + (int)rank * 128 + row_local;
+            float* sk_row = kind == 0 ? nullptr
+                          : p.sk_partial + (size_t)slot * SK_SLOT_FLOATS + ((size_t)rank * 128 + row_local) * 256;
             epilogue_segment<MODE>(p, gi, tile.y, row, tile.w * S2_BN,
-                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * 128);
+                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * 128, kind, sk_row,
+                                   nsl);
             tc_fence_before();
+            if (kind == 2) __threadfence();
             __syncwarp();
-            if (lane == 0) mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
+            if (lane == 0) {
+                if (kind == 2 && atomicAdd(&p.sk_count[slot], 1) == 2 * NUM_EPI_WARPS - 1) {
+                    // last of the 16 epilogue warps of the pair: the slot is complete
+                    p.sk_count[slot] = 0;
+                    __threadfence();
+                    st_release_gpu(&p.sk_flag[slot], p.epoch);
+                }
+                mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
+            }
         }
     }
 

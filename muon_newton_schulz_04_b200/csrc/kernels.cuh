@@ -76,7 +76,23 @@ struct GemmParams {
     const float* scale;           // per-matrix 1/(||U||+eps) on the first iteration, else nullptr
     int write_op;                 // UPDATE: also write the bf16 operand copy of X'
     int* err;                     // device error word (bounded waits)
+    // UPDATE of the last iteration only: 1 = also apply W <- decay*W - lr*s*O,
+    // 2 = also copy O out to the caller (orthogonalisation), 0 = neither.
+    int apply_mode;
+    float decay, lr;
+    const EwSeg* segs;            // per-matrix W / output pointer, orientation and scale
+    // two-CTA kernel: per-cluster work units (see plan.h), two int4 per unit:
+    // (group, matrix, tile_row, tile_col) and (k_begin, k_end, kind, slot | nslots << 16)
+    const int4* units;
+    const int* unit_begin;        // clusters + 1 offsets
+    float* sk_partial;            // partial-sum slots, SK_SLOT_FLOATS each
+    int* sk_count;                // per slot: epilogue warps that have stored their part
+    int* sk_flag;                 // per slot: epoch of the last complete partial
+    int epoch;                    // distinct per launch on a handle
 };
+
+// One partial-sum slot: both CTAs' 128 x 256 fp32 accumulator halves.
+constexpr int SK_SLOT_FLOATS = 2 * 128 * 256;
 
 // pair = 1: the two-CTA kernel (256 x 256 tiles, grid = 2 x clusters);
 // pair = 0: the one-CTA kernel (128 x 256 tiles).
@@ -106,9 +122,10 @@ struct SimtGemmArgs {
 cudaError_t launch_simt_gemm(const SimtGemmArgs& a, cudaStream_t s);
 
 // Elementwise kernels.
+// Momentum, Nesterov direction, oriented X0 and, per matrix, ||U||_F and
+// s = 1/(||U||_F + eps).  counters: one int per matrix, zero between calls.
 cudaError_t launch_momentum_norm(const EwSeg* segs, int nseg, int nblocks, double* partials,
-                                 float mu, int nesterov, int bf16_operand, cudaStream_t s);
-cudaError_t launch_norm_finalize(const EwSeg* segs, int nseg, const double* partials, float eps,
+                                 float mu, int nesterov, int bf16_operand, int* counters, float eps,
                                  float* norms, float* scale, cudaStream_t s);
 cudaError_t launch_apply(const EwSeg* segs, int nseg, int nblocks, float decay, float lr,
                          const float* o_scale, int copy_out, cudaStream_t s);

@@ -52,6 +52,67 @@ std::vector<Tile> build_tiles(const std::vector<GroupDims>& groups, int phase, i
     return out;
 }
 
+UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kblocks, int clusters, bool split) {
+    UnitPlan up;
+    const int T = (int)tiles.size();
+    const int C = clusters < 1 ? 1 : clusters;
+    const int R = split ? T % C : 0;
+    const int D = T - R;
+    std::vector<std::vector<Unit>> per(C);
+    for (int t = 0; t < D; ++t) per[t % C].push_back(Unit{tiles[t], 0, kblocks[t], 0, 0, 0});
+    if (R > 0) {
+        // flatten the remaining tiles' K-blocks and cut them into C ranges
+        long long total = 0;
+        std::vector<long long> start(R + 1, 0);
+        for (int r = 0; r < R; ++r) { start[r] = total; total += kblocks[D + r]; }
+        start[R] = total;
+        std::vector<std::vector<Unit>> sk(C);
+        std::vector<std::vector<int>> tile_units(R);     // (cluster) of each part, in K order
+        std::vector<std::vector<int>> tile_pos(R);
+        for (int c = 0; c < C; ++c) {
+            long long a = total * c / C, b = total * (c + 1) / C;
+            int r = 0;
+            while (r < R && start[r + 1] <= a) ++r;
+            while (a < b && r < R) {
+                const long long e = std::min(b, start[r + 1]);
+                const int kb = (int)(a - start[r]), ke = (int)(e - start[r]);
+                tile_units[r].push_back(c);
+                tile_pos[r].push_back((int)sk[c].size());
+                sk[c].push_back(Unit{tiles[D + r], kb, ke, kb == 0 ? 1 : 2, 0, 0});
+                a = e;
+                ++r;
+            }
+        }
+        int slot = 0;
+        for (int r = 0; r < R; ++r) {
+            const int n = (int)tile_units[r].size();
+            if (n == 1) { sk[tile_units[r][0]][tile_pos[r][0]].kind = 0; continue; }
+            Unit& head = sk[tile_units[r][0]][tile_pos[r][0]];
+            head.kind = 1;
+            head.slot = slot;
+            head.nslots = n - 1;
+            for (int i = 1; i < n; ++i) {
+                Unit& part = sk[tile_units[r][i]][tile_pos[r][i]];
+                part.kind = 2;
+                part.slot = slot++;
+            }
+        }
+        up.nslots = slot;
+        for (int c = 0; c < C; ++c) per[c].insert(per[c].end(), sk[c].begin(), sk[c].end());
+    }
+    up.begin.push_back(0);
+    for (int c = 0; c < C; ++c) {
+        up.units.insert(up.units.end(), per[c].begin(), per[c].end());
+        up.begin.push_back((int)up.units.size());
+    }
+    return up;
+}
+
+int tc_gemm_split_tiles() {
+    const char* v = std::getenv("MUON_GEMM_SPLIT");
+    return (v && std::strcmp(v, "1") == 0) ? 1 : 0;
+}
+
 int tc_gemm_default_pair() {
     const char* v = std::getenv("MUON_GEMM_PAIR");
     return (v && std::strcmp(v, "0") == 0) ? 0 : 1;

@@ -26,6 +26,34 @@ GroupDims make_dims(int rows, int cols, int count);
 // descending, ties in (group, matrix, tile_row, tile_col) order.
 std::vector<Tile> build_tiles(const std::vector<GroupDims>& groups, int phase, int bm, int bn);
 
+// Work units of the persistent two-CTA kernel.  Each unit is a tile and a K-block
+// range [k_begin, k_end) of it:
+//   kind 0: the whole tile, finished by its unit;
+//   kind 1: the head of a split tile (k_begin = 0): adds the fp32 partial sums of
+//           slots [slot, slot + nslots) after its own range, then finishes the tile;
+//   kind 2: a later part of a split tile: writes its fp32 partial sum to `slot`.
+// Units are listed per cluster in execution order; cluster c runs
+// units[begin[c] .. begin[c+1]).  The tiles of full rounds (floor(T / C) * C of them,
+// T tiles, C clusters) are whole units dealt round-robin; when split is true and
+// T % C != 0, the K-blocks of the remaining tiles are divided into C contiguous,
+// nearly equal ranges, one per cluster, so every cluster ends at about the same
+// time.  A cluster's range starts with at most one kind-2 unit, so a head unit only
+// waits for partials that their clusters produce before doing anything else.
+struct Unit { Tile tile; int k_begin, k_end, kind, slot, nslots; };
+
+struct UnitPlan {
+    std::vector<Unit> units;
+    std::vector<int> begin;   // C + 1 offsets
+    int nslots = 0;           // partial-sum slots used
+};
+
+UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kblocks, int clusters, bool split);
+
+// 0 unless the environment variable MUON_GEMM_SPLIT is "1": split the K-blocks of
+// the last, partial round of tiles over all clusters (build_units).  Off by
+// default: on the 4096 x 4096 workload it measured slower than whole tiles.
+int tc_gemm_split_tiles();
+
 // 1 unless the environment variable MUON_GEMM_PAIR is "0" (see kernels.cuh).
 int tc_gemm_default_pair();
 

@@ -162,3 +162,47 @@ def test_symmetric_tiles_skip_the_lower_triangle():
     sym = len(mb.plan_tiles([(4096, 4096, 1)], 0))
     assert full == (4096 // BM) * (4096 // BN)
     assert sym < 0.56 * full
+
+
+@pytest.mark.parametrize("shapes,clusters", [([(4096, 4096, 1)], 74), ([(4096, 4096, 1)], 5), ([(256, 512, 1)], 74),
+                                             ([(768, 768, 4), (3072, 768, 1)], 74), ([(2048, 1408, 3)], 74),
+                                             ([(1024, 1536, 1)], 74), ([(1600, 1600, 2), (6400, 1600, 1)], 74)])
+@pytest.mark.parametrize("phase", [0, 1, 2])
+def test_units_cover_each_k_block_once_and_never_chain_waits(shapes, clusters, phase):
+    units = mb.plan_units(shapes, phase, clusters)
+    tiles = mb.plan_tiles(shapes, phase)
+    dims = [(min(r, c), max(r, c)) for (r, c, _) in shapes]
+    kbl = {t: ((dims[t[0]][1] if phase == 0 else dims[t[0]][0]) + 63) // 64 for t in tiles}
+    seen = {t: [] for t in tiles}
+    by_cluster = {}
+    slots = {}
+    for (c, g, z, tr, tc, kb, ke, kind, slot, nsl) in units:
+        seen[(g, z, tr, tc)].append((kb, ke, kind, slot, nsl, c))
+        by_cluster.setdefault(c, []).append(kind)
+        if kind == 2:
+            assert slot not in slots
+            slots[slot] = (g, z, tr, tc, kb)
+    for t, parts in seen.items():
+        parts.sort()
+        assert parts, t
+        cover = [(kb, ke) for (kb, ke, *_r) in parts]
+        assert cover[0][0] == 0 and cover[-1][1] == kbl[t]
+        assert all(cover[i][1] == cover[i + 1][0] for i in range(len(cover) - 1))     # contiguous, no overlap
+        if len(parts) == 1:
+            assert parts[0][2] == 0
+        else:
+            head = parts[0]
+            assert head[2] == 1 and head[4] == len(parts) - 1
+            for i, p in enumerate(parts[1:]):
+                assert p[2] == 2 and p[3] == head[3] + i                            # slots in K order
+                assert p[5] != head[5]                                              # another cluster
+    for c, kinds in by_cluster.items():
+        # a waiting head is its cluster's last unit and each cluster produces at most one
+        # partial, before any wait: producers never wait, so waits cannot chain
+        assert all(k != 1 for k in kinds[:-1]) and kinds.count(2) <= 1
+    assert set(c for (c, *_r) in units) <= set(range(clusters))
+
+
+def test_no_undefined_library_symbols():
+    out = os.popen(f"nm -D --undefined-only {mb.LIB_PATH}").read()
+    assert "muon" not in out

@@ -15,21 +15,22 @@ from muon_newton_schulz_04_b200 import build as mbuild
 pytestmark = pytest.mark.gpu
 
 
-@pytest.fixture(scope="module", params=["pair", "single"])
+@pytest.fixture(scope="module", params=["pair", "pair-split", "single"])
 def opt(request):
-    """A handle on the two-CTA GEMM kernel (default) and one on the one-CTA kernel."""
+    """Handles on the two-CTA GEMM kernel (default), the two-CTA kernel with the last
+    round of tiles split over all clusters, and the one-CTA kernel."""
     mbuild.build()
-    old = os.environ.get("MUON_GEMM_PAIR")
-    os.environ["MUON_GEMM_PAIR"] = "1" if request.param == "pair" else "0"
-    try:
-        o = mb.Muon(mb.config())
-    finally:
-        if old is None:
-            del os.environ["MUON_GEMM_PAIR"]
-        else:
-            os.environ["MUON_GEMM_PAIR"] = old
+    env = {"pair": ("1", "0"), "pair-split": ("1", "1"), "single": ("0", "0")}[request.param]
+    old = {k: os.environ.get(k) for k in ("MUON_GEMM_PAIR", "MUON_GEMM_SPLIT")}
+    os.environ["MUON_GEMM_PAIR"], os.environ["MUON_GEMM_SPLIT"] = env
+    o = mb.Muon(mb.config())
     yield o
     o.close()
+    for k, v in old.items():
+        if v is None:
+            os.environ.pop(k, None)
+        else:
+            os.environ[k] = v
 
 
 def bf16(x: np.ndarray) -> torch.Tensor:
