@@ -17,6 +17,7 @@
 // vectors); tall matrices go through a 64x64 shared-memory transpose so that
 // both the row-major reads and the transposed writes stay coalesced.
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace muon {
 namespace {
@@ -63,6 +64,8 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* 
                                                                   float* __restrict__ norms, float* __restrict__ scale) {
     __shared__ float tile[EW_TILE][EW_TILE + 1];
     __shared__ double red[EW_THREADS / 32];
+    pdl_trigger();
+    pdl_wait();
     const int si = find_seg(segs, nseg, blockIdx.x, false);
     const EwSeg sg = segs[si];
     const int lb = blockIdx.x - sg.blk_begin;
@@ -237,12 +240,16 @@ __device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay
 
 __global__ void __launch_bounds__(EW_THREADS) apply_kernel(const EwSeg* __restrict__ segs, int nseg, float decay,
                                                           float lr, const float* __restrict__ o_scale, int copy_out) {
+    pdl_trigger();
+    pdl_wait();
     const int si = find_seg(segs, nseg, blockIdx.x, true);
     const EwSeg sg = segs[si];
     apply_block(sg, blockIdx.x - sg.apply_begin, decay, lr, o_scale, copy_out, sg.w);
 }
 
 __global__ void __launch_bounds__(EW_THREADS) copy_out_one_kernel(const EwSeg sg, float* dst, const float* o_scale) {
+    pdl_trigger();
+    pdl_wait();
     apply_block(sg, blockIdx.x, 1.0f, 0.0f, o_scale, 1, dst);
 }
 
@@ -252,22 +259,19 @@ cudaError_t launch_momentum_norm(const EwSeg* segs, int nseg, int nblocks, doubl
                                  int nesterov, int bf16_operand, int* counters, float eps, float* norms,
                                  float* scale, cudaStream_t s) {
     if (nblocks <= 0) return cudaSuccess;
-    momentum_norm_kernel<<<nblocks, EW_THREADS, 0, s>>>(segs, nseg, partials, mu, nesterov, bf16_operand, counters,
-                                                        eps, norms, scale);
-    return cudaGetLastError();
+    return launch_pdl(momentum_norm_kernel, dim3(nblocks), dim3(EW_THREADS), 0, s, segs, nseg, partials, mu, nesterov,
+                      bf16_operand, counters, eps, norms, scale);
 }
 
 cudaError_t launch_apply(const EwSeg* segs, int nseg, int nblocks, float decay, float lr, const float* o_scale,
                          int copy_out, cudaStream_t s) {
     if (nblocks <= 0) return cudaSuccess;
-    apply_kernel<<<nblocks, EW_THREADS, 0, s>>>(segs, nseg, decay, lr, o_scale, copy_out);
-    return cudaGetLastError();
+    return launch_pdl(apply_kernel, dim3(nblocks), dim3(EW_THREADS), 0, s, segs, nseg, decay, lr, o_scale, copy_out);
 }
 
 cudaError_t launch_copy_out_one(const EwSeg& seg, float* dst, const float* o_scale, cudaStream_t s) {
     if (seg.apply_count <= 0) return cudaSuccess;
-    copy_out_one_kernel<<<seg.apply_count, EW_THREADS, 0, s>>>(seg, dst, o_scale);
-    return cudaGetLastError();
+    return launch_pdl(copy_out_one_kernel, dim3(seg.apply_count), dim3(EW_THREADS), 0, s, seg, dst, o_scale);
 }
 
 }  // namespace muon

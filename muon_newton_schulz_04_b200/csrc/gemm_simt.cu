@@ -7,6 +7,7 @@
 // C[z] = alpha_eff * A[z] op(B[z]) + beta_eff * Cin[z], 64x64 output tile per
 // block, 256 threads with a 4x4 register tile each, K staged 16 at a time.
 #include "kernels.cuh"
+#include "ptx.cuh"
 
 namespace muon {
 namespace {
@@ -16,6 +17,8 @@ constexpr int SB = 64, SK = 16;
 __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtGemmArgs a) {
     __shared__ float As[SK][SB + 4];
     __shared__ float Bs[SK][SB + 4];
+    pdl_trigger();
+    pdl_wait();
     const int z = blockIdx.z;
     const int i0 = blockIdx.y * SB, j0 = blockIdx.x * SB;
     const float* A = a.A + (size_t)z * a.sA;
@@ -80,8 +83,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtGemmArgs a) {
 cudaError_t launch_simt_gemm(const SimtGemmArgs& a, cudaStream_t s) {
     if (a.M <= 0 || a.N <= 0 || a.count <= 0) return cudaSuccess;
     dim3 grid((a.N + SB - 1) / SB, (a.M + SB - 1) / SB, a.count);
-    simt_gemm_kernel<<<grid, 256, 0, s>>>(a);
-    return cudaGetLastError();
+    return launch_pdl(simt_gemm_kernel, grid, dim3(256), 0, s, a);
 }
 
 }  // namespace muon

@@ -355,6 +355,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger();
+    pdl_wait();             // operands and outputs belong to the previous kernels
 
     if (warp == 0) {
         if (elect_one()) {
@@ -514,6 +516,8 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
     cluster_sync_all();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_trigger();
+    pdl_wait();             // operands and outputs belong to the previous kernels
 
     if (warp == 0) {
         if (elect_one()) {
@@ -679,20 +683,19 @@ cudaError_t tc_gemm_max_clusters(int* n) {
 
 cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cudaStream_t s) {
     if (p.ntiles <= 0) return cudaSuccess;
+    const dim3 g(grid), b(NUM_THREADS);
     if (pair) {
         switch (mode) {
-            case MODE_GRAM: ns_gemm_tc2_kernel<MODE_GRAM><<<grid, NUM_THREADS, S2_SMEM, s>>>(p); break;
-            case MODE_POLY: ns_gemm_tc2_kernel<MODE_POLY><<<grid, NUM_THREADS, S2_SMEM, s>>>(p); break;
-            default: ns_gemm_tc2_kernel<MODE_UPDATE><<<grid, NUM_THREADS, S2_SMEM, s>>>(p); break;
-        }
-    } else {
-        switch (mode) {
-            case MODE_GRAM: ns_gemm_tc_kernel<MODE_GRAM><<<grid, NUM_THREADS, S1_SMEM, s>>>(p); break;
-            case MODE_POLY: ns_gemm_tc_kernel<MODE_POLY><<<grid, NUM_THREADS, S1_SMEM, s>>>(p); break;
-            default: ns_gemm_tc_kernel<MODE_UPDATE><<<grid, NUM_THREADS, S1_SMEM, s>>>(p); break;
+            case MODE_GRAM: return launch_pdl(ns_gemm_tc2_kernel<MODE_GRAM>, g, b, S2_SMEM, s, p);
+            case MODE_POLY: return launch_pdl(ns_gemm_tc2_kernel<MODE_POLY>, g, b, S2_SMEM, s, p);
+            default: return launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE>, g, b, S2_SMEM, s, p);
         }
     }
-    return cudaGetLastError();
+    switch (mode) {
+        case MODE_GRAM: return launch_pdl(ns_gemm_tc_kernel<MODE_GRAM>, g, b, S1_SMEM, s, p);
+        case MODE_POLY: return launch_pdl(ns_gemm_tc_kernel<MODE_POLY>, g, b, S1_SMEM, s, p);
+        default: return launch_pdl(ns_gemm_tc_kernel<MODE_UPDATE>, g, b, S1_SMEM, s, p);
+    }
 }
 
 }  // namespace muon

@@ -131,6 +131,24 @@ cudaError_t launch_apply(const EwSeg* segs, int nseg, int nblocks, float decay, 
                          const float* o_scale, int copy_out, cudaStream_t s);
 cudaError_t launch_copy_out_one(const EwSeg& seg, float* dst, const float* o_scale, cudaStream_t s);
 
+// Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger in
+// ptx.cuh): the kernel may start while the previous kernel of the stream drains and
+// waits on the device before it touches that kernel's data.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 constexpr int EW_THREADS = 256;
 constexpr int EW_FLAT_ELEMS = 8192;      // elements per block on the flat path
 constexpr int EW_TILE = 64;              // transpose tile edge

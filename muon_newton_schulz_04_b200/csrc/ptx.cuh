@@ -277,3 +277,17 @@ __device__ __forceinline__ void tc_commit_pair(uint32_t bar_cluster_addr) {
 }
 
 }  // namespace muon
+
+// ---------------------------------------------------------------- programmatic dependent launch
+// Kernels of the step are launched with programmatic stream serialisation: the next
+// kernel may be scheduled while this one drains.  Each kernel does its set-up
+// (barriers, TMEM, descriptor prefetch) first, then waits for the previous grid to
+// complete before it reads or writes any data that grid touches.  Without the launch
+// attribute both instructions are no-ops.
+namespace muon {
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+}  // namespace muon
