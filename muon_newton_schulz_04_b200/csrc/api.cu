@@ -9,6 +9,7 @@
 // All launches go to the caller's stream; nothing here synchronises except the
 // entry points documented to do so.
 #include <cmath>
+#include <cstdlib>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -67,6 +68,7 @@ struct Plan {
     float* d_scale = nullptr;
     int* d_counters = nullptr;           // per-matrix block counters of the momentum kernel
     bool valid = false;
+    unsigned long long version = 0;      // distinct per built plan
     std::vector<EwSeg> uploaded;         // last segment table copied to the device
 };
 
@@ -96,6 +98,17 @@ struct muon_handle {
     int t_n[MUON_TIMING_KINDS] = {};
     // muon_step_host: side stream for copies that overlap the GEMMs, and its events
     cudaStream_t side = nullptr;
+    // captured launch sequence of muon_step / muon_orthogonalize (replayed while the
+    // plan, the caller's pointers and the configuration stay the same)
+    bool graphs = true;
+    cudaStream_t cap_stream = nullptr;
+    cudaGraphExec_t gexec = nullptr;
+    std::vector<EwSeg> g_segs;
+    muon_config g_cfg;
+    void* g_ws = nullptr;
+    int g_mode = -1;
+    unsigned long long g_version = 0;
+    unsigned long long plans_built = 0;
     cudaEvent_t ev_start = nullptr, ev_w = nullptr, ev_k1 = nullptr, ev_done = nullptr;
 };
 
@@ -280,6 +293,7 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
     if (P.valid && P.key == key) return MUON_OK;
     P = Plan();
     P.key = key;
+    P.version = ++h->plans_built;
     const bool bf16 = is_bf16_path(h);
     const int ng = (int)shapes.size() / 3;
     size_t off = 0;
@@ -568,6 +582,44 @@ muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStrea
     return MUON_OK;
 }
 
+// Replays the captured launch sequence when nothing it depends on has changed,
+// else captures it again on a private stream (graph capture is not allowed on the
+// legacy default stream).  Direct launches when timing is on, when the host-buffer
+// step splices copies in, when the caller's stream is itself being captured, or when
+// split tiles are used (their flags carry a per-launch epoch).
+muon_status run_graph_or_direct(muon_handle* h, bool momentum, bool copy_out, cudaStream_t s, const Hooks* hooks) {
+    Plan& P = h->plan;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    CUDA_TRY(h, cudaStreamIsCapturing(s, &cs));
+    const bool use_graph = h->graphs && !h->timing && !hooks && cs == cudaStreamCaptureStatusNone &&
+                           !(h->pair && tc_gemm_split_tiles());
+    if (!use_graph) return run_pipeline(h, momentum, copy_out, s, hooks);
+    const int mode = copy_out ? 1 : 0;
+    const bool same = h->gexec && h->g_mode == mode && h->g_ws == h->ws.ptr && h->g_version == P.version &&
+                      std::memcmp(&h->g_cfg, &h->cfg, sizeof(muon_config)) == 0 && h->g_segs.size() == P.uploaded.size() &&
+                      std::memcmp(h->g_segs.data(), P.uploaded.data(), P.uploaded.size() * sizeof(EwSeg)) == 0;
+    if (!same) {
+        if (h->gexec) { cudaGraphExecDestroy(h->gexec); h->gexec = nullptr; }
+        if (!h->cap_stream) CUDA_TRY(h, cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking));
+        CUDA_TRY(h, cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
+        muon_status st = run_pipeline(h, momentum, copy_out, h->cap_stream, nullptr);
+        cudaGraph_t graph = nullptr;
+        cudaError_t e = cudaStreamEndCapture(h->cap_stream, &graph);
+        if (st != MUON_OK) { if (graph) cudaGraphDestroy(graph); return st; }
+        if (e != cudaSuccess) return fail(h, MUON_ERR_CUDA, "graph capture failed: %s", cudaGetErrorString(e));
+        e = cudaGraphInstantiate(&h->gexec, graph, 0);
+        cudaGraphDestroy(graph);
+        if (e != cudaSuccess) { h->gexec = nullptr; return fail(h, MUON_ERR_CUDA, "graph instantiation failed: %s", cudaGetErrorString(e)); }
+        h->g_mode = mode;
+        h->g_ws = h->ws.ptr;
+        h->g_version = P.version;
+        h->g_cfg = h->cfg;
+        h->g_segs = P.uploaded;
+    }
+    CUDA_TRY(h, cudaGraphLaunch(h->gexec, s));
+    return MUON_OK;
+}
+
 muon_status step_device(muon_handle* h, const muon_group* groups, int n, cudaStream_t s,
                         const Hooks* hooks = nullptr) {
     std::vector<int> shapes;
@@ -581,7 +633,7 @@ muon_status step_device(muon_handle* h, const muon_group* groups, int n, cudaStr
     muon_status st = ensure_plan(h, shapes, s);
     if (st != MUON_OK) return st;
     if ((st = upload_segs(h, mp, s)) != MUON_OK) return st;
-    return run_pipeline(h, true, false, s, hooks);
+    return run_graph_or_direct(h, true, false, s, hooks);
 }
 
 }  // namespace
@@ -632,6 +684,10 @@ muon_status muon_create(const muon_config* cfg, int device, muon_handle** out) {
     h->device = device;
     h->num_sms = prop.multiProcessorCount;
     h->pair = tc_gemm_default_pair();
+    {
+        const char* v = std::getenv("MUON_GRAPHS");
+        h->graphs = !(v && std::strcmp(v, "0") == 0);
+    }
     DeviceGuard dg(device);
     if (cudaMalloc(&h->d_err, sizeof(int)) != cudaSuccess || cudaMemset(h->d_err, 0, sizeof(int)) != cudaSuccess) {
         cudaGetLastError();
@@ -764,7 +820,7 @@ muon_status muon_orthogonalize(muon_handle* h, const muon_ortho_group* groups, i
     muon_status st = ensure_plan(h, shapes, s);
     if (st != MUON_OK) return st;
     if ((st = upload_segs(h, mp, s)) != MUON_OK) return st;
-    return run_pipeline(h, false, true, s);
+    return run_graph_or_direct(h, false, true, s, nullptr);
 }
 
 muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void* stream) {
@@ -969,6 +1025,8 @@ muon_status muon_destroy(muon_handle* h) {
         cudaEvent_t evs[4] = {h->ev_start, h->ev_w, h->ev_k1, h->ev_done};
         for (cudaEvent_t e : evs) if (e) cudaEventDestroy(e);
         if (h->side) cudaStreamDestroy(h->side);
+        if (h->gexec) cudaGraphExecDestroy(h->gexec);
+        if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
         if (h->ws.ptr) cudaFree(h->ws.ptr);
         if (h->staging.ptr) cudaFree(h->staging.ptr);
         if (h->scratch.ptr) cudaFree(h->scratch.ptr);
