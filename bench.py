@@ -142,11 +142,11 @@ class ClockSampler:
 def elementwise_bytes(w: wl.Workload):
     """Algorithmic HBM bytes of the two memory-bound kernels of one step.
 
-    momentum+norm: read G (2 or 4 B) and B (4 B), write B (4 B), the fp32 iterate
-    (4 B) and its bf16 operand copy (2 B) = 16 B/elem for bf16 gradients.
-    apply: read W (4 B) and the fp32 result O (4 B), write W (4 B) = 12 B/elem."""
+    momentum+norm: read G (2 or 4 B) and B (4 B), write B (4 B) and the iterate as
+    a bf16 pair hi + lo (2 + 2 B) = 14 B/elem for bf16 gradients.
+    apply (when not fused): read W (4 B) and O = hi + lo (4 B), write W (4 B) = 12 B/elem."""
     g = 2 if w.grad_dtype == wl.BF16 else 4
-    return w.elements * (g + 4 + 4 + 4 + 2), w.elements * 12
+    return w.elements * (g + 4 + 4 + 2 + 2), w.elements * 12
 
 
 def update_gemm_flops(w: wl.Workload):
@@ -379,7 +379,7 @@ def run_ours(args, w):
     d2h = w.elements * (4 + 4)
 
     ws_bytes = w.elements * (4 + 4 + gbytes) + sum(
-        min(s.rows, s.cols) * (max(s.rows, s.cols) * (2 + 2 + 4) + 2 * 2 * min(s.rows, s.cols)) for s in w.matrices)
+        min(s.rows, s.cols) * (max(s.rows, s.cols) * (2 + 2 + 2) + 2 * 2 * min(s.rows, s.cols)) for s in w.matrices)
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",

@@ -56,8 +56,9 @@ typedef enum {
 
 typedef enum { MUON_BF16 = 0, MUON_FP32 = 1 } muon_dtype;
 
-/* MUON_PREC_BF16: tensor-core GEMMs with bf16 operands and fp32 accumulation, the
- *   iterate X additionally carried in fp32 for the aX term (the timed path).
+/* MUON_PREC_BF16: tensor-core GEMMs with bf16 operands and fp32 accumulation; the
+ *   iterate X is carried as a pair of bf16 arrays X = hi + lo (about 16 significant
+ *   bits) so that the aX term keeps that precision (the timed path).
  * MUON_PREC_FP32_DEBUG: every Newton-Schulz GEMM in fp32 FFMA (no TF32). */
 typedef enum { MUON_PREC_BF16 = 0, MUON_PREC_FP32_DEBUG = 1 } muon_precision;
 
@@ -140,16 +141,19 @@ muon_status muon_orthogonalize(muon_handle* h, const muon_ortho_group* groups, i
 /* One Newton-Schulz building block on caller buffers, for per-kernel checks and
  * for callers composing their own iteration (section 4 eq. 4 grouped as
  * A = XX^T, P = bA + cA^2, X' = aX + PX).  All buffers are device memory, densely
- * packed [count][rows][cols].  With precision BF16, m and n must be multiples of 8.
+ * packed [count][rows][cols], 16-byte aligned.  With precision BF16, m and n must
+ * be multiples of 8.
  *
  *  MUON_NS_GRAM:   out(m x m)   = alpha * X X^T            X = x_op (m x n)
  *  MUON_NS_POLY:   out(m x m)   = beta * A + alpha * A A   A = a_in (m x m, symmetric)
- *  MUON_NS_UPDATE: out(m x n)   = alpha * P X + beta * Xm   P = a_in (m x m), X = x_op,
- *                                                          Xm = x_master (fp32, m x n)
- *                  and, if out_op != NULL, out_op = bf16(out)   (BF16 precision only)
+ *  MUON_NS_UPDATE: X'(m x n)    = alpha * P X + beta * X   P = a_in (m x m)
  *
- * Types: BF16 precision: x_op, a_in and the GRAM/POLY out are bf16; UPDATE out
- * and x_master are fp32.  FP32_DEBUG precision: every buffer is fp32. */
+ * BF16 precision: x_op, a_in and the GRAM / POLY out are bf16.  The iterate of
+ * UPDATE is a pair of bf16 arrays, X = x_op + x_master (high part, which is also
+ * the GEMM operand, and low part); the result is written the same way,
+ * X' = out + out_op with out = bf16(X') and out_op = bf16(X' - out).
+ * FP32_DEBUG precision: every buffer is fp32; UPDATE reads X = x_op for the
+ * product and x_master for the beta term, and writes X' to out. */
 typedef enum { MUON_NS_GRAM = 0, MUON_NS_POLY = 1, MUON_NS_UPDATE = 2 } muon_ns_phase;
 
 typedef struct {
@@ -159,7 +163,7 @@ typedef struct {
     float alpha, beta;
     const void* x_op;
     const void* a_in;
-    const float* x_master;
+    const void* x_master;
     void* out;
     void* out_op;
 } muon_ns_phase_args;

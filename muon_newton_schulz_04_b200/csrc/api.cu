@@ -38,7 +38,7 @@ struct DevBuf {
 
 // Workspace offsets of one group (bytes from the workspace base).
 struct GroupOffsets {
-    size_t xb[2], xf[2], a, p;
+    size_t xb[2], xl, xf[2], a, p;
 };
 
 struct Plan {
@@ -307,10 +307,11 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
         const size_t xe = (size_t)d.count * d.m * d.ldn, ae = (size_t)d.count * d.m * d.ldm;
         if (bf16) {
             o.xb[0] = take(xe * 2); o.xb[1] = take(xe * 2);
-            o.xf[0] = take(xe * 4); o.xf[1] = o.xf[0];
+            o.xl = take(xe * 2);
+            o.xf[0] = o.xf[1] = 0;
             o.a = take(ae * 2); o.p = take(ae * 2);
         } else {
-            o.xb[0] = o.xb[1] = 0;
+            o.xb[0] = o.xb[1] = o.xl = 0;
             o.xf[0] = take(xe * 4); o.xf[1] = take(xe * 4);
             o.a = take(ae * 4); o.p = take(ae * 4);
         }
@@ -405,8 +406,12 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
         const size_t xe = (size_t)d.m * d.ldn;
         for (int z = 0; z < d.count; ++z, ++mi) {
             EwSeg& sg = P.segs[mi];
-            sg.xf0 = reinterpret_cast<float*>(base + P.offs[g].xf[0]) + (size_t)z * xe;
-            sg.xb0 = bf16 ? static_cast<void*>(reinterpret_cast<__nv_bfloat16*>(base + P.offs[g].xb[0]) + (size_t)z * xe) : nullptr;
+            if (bf16) {
+                sg.xhi0 = reinterpret_cast<__nv_bfloat16*>(base + P.offs[g].xb[0]) + (size_t)z * xe;
+                sg.xlo0 = reinterpret_cast<__nv_bfloat16*>(base + P.offs[g].xl) + (size_t)z * xe;
+            } else {
+                sg.xf0 = reinterpret_cast<float*>(base + P.offs[g].xf[0]) + (size_t)z * xe;
+            }
         }
     }
     if (bf16) {
@@ -426,8 +431,8 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
             q.m = d.m; q.n = d.n; q.ldm = d.ldm; q.ldn = d.ldn; q.count = d.count; q.mat_base = P.mat_base[g];
             q.xb[0] = reinterpret_cast<__nv_bfloat16*>(base + o.xb[0]);
             q.xb[1] = reinterpret_cast<__nv_bfloat16*>(base + o.xb[1]);
-            q.xf_in = reinterpret_cast<const float*>(base + o.xf[0]);
-            q.xf_out = reinterpret_cast<float*>(base + o.xf[0]);
+            q.xlo_in = reinterpret_cast<const __nv_bfloat16*>(base + o.xl);
+            q.xlo_out = reinterpret_cast<__nv_bfloat16*>(base + o.xl);
             q.a = reinterpret_cast<__nv_bfloat16*>(base + o.a);
             q.p = reinterpret_cast<__nv_bfloat16*>(base + o.p);
         }
@@ -487,7 +492,12 @@ muon_status upload_segs(muon_handle* h, const std::vector<MatPtrs>& mp, cudaStre
             sg.g = mp[mi].g; sg.b = mp[mi].b; sg.w = mp[mi].w;
             sg.g_bf16 = mp[mi].g_bf16;
             sg.update_scale = mp[mi].scale;
-            sg.o_src = reinterpret_cast<const float*>(base + P.offs[g].xf[final_buf]) + (size_t)z * xe;
+            if (bf16) {
+                sg.o_hi = reinterpret_cast<const __nv_bfloat16*>(base + P.offs[g].xb[h->cfg.ns_steps & 1]) + (size_t)z * xe;
+                sg.o_lo = reinterpret_cast<const __nv_bfloat16*>(base + P.offs[g].xl) + (size_t)z * xe;
+            } else {
+                sg.o_src = reinterpret_cast<const float*>(base + P.offs[g].xf[final_buf]) + (size_t)z * xe;
+            }
             sg.vec = (d.cols % 8 == 0) && aligned(sg.g, 16) && aligned(sg.w, 16) && (sg.b == nullptr || aligned(sg.b, 16)) ? 1 : 0;
         }
     }
@@ -835,6 +845,8 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     if (a->phase != MUON_NS_POLY && !a->x_op) return fail(h, MUON_ERR_INVALID, "x_op is NULL");
     if (a->phase != MUON_NS_GRAM && !a->a_in) return fail(h, MUON_ERR_INVALID, "a_in is NULL");
     if (a->phase == MUON_NS_UPDATE && !a->x_master) return fail(h, MUON_ERR_INVALID, "x_master is NULL");
+    if (a->phase == MUON_NS_UPDATE && a->precision == MUON_PREC_BF16 && !a->out_op)
+        return fail(h, MUON_ERR_INVALID, "out_op (low part of the result) is NULL");
     const bool bf16 = a->precision == MUON_PREC_BF16;
     if (bf16 && (a->m % 8 != 0 || a->n % 8 != 0)) return fail(h, MUON_ERR_UNSUPPORTED, "bf16 building blocks need m and n multiples of 8");
     const void* ptrs[5] = {a->x_op, a->a_in, a->x_master, a->out, a->out_op};
@@ -855,7 +867,8 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
             g.A = (const float*)a->a_in; g.B = (const float*)a->a_in; g.C = (float*)a->out; g.Cin = (const float*)a->a_in;
             g.M = m; g.N = m; g.K = m; g.lda = g.ldb = g.ldc = g.ldcin = m; g.sA = g.sB = g.sC = g.sCin = (long long)m * m; g.b_kmajor = 1;
         } else {
-            g.A = (const float*)a->a_in; g.B = (const float*)a->x_op; g.C = (float*)a->out; g.Cin = a->x_master;
+            g.A = (const float*)a->a_in; g.B = (const float*)a->x_op; g.C = (float*)a->out;
+            g.Cin = (const float*)a->x_master;
             g.M = m; g.N = n; g.K = m; g.lda = m; g.ldb = n; g.ldc = n; g.ldcin = n;
             g.sA = (long long)m * m; g.sB = g.sC = g.sCin = (long long)m * n; g.b_kmajor = 0;
         }
@@ -889,9 +902,10 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     } else {
         if ((st = encode_map(h, &maps.p, a->a_in, m, m, cnt, m, 128)) != MUON_OK) return st;
         if ((st = encode_map(h, &maps.xb_mn[0], a->x_op, n, m, cnt, n, 64)) != MUON_OK) return st;
-        gi.xf_in = a->x_master;
-        gi.xf_out = (float*)a->out;
-        gi.xb[1] = (__nv_bfloat16*)a->out_op;
+        gi.xb[0] = (__nv_bfloat16*)a->x_op;            // X = x_op + x_master (high + low part)
+        gi.xlo_in = (const __nv_bfloat16*)a->x_master;
+        gi.xb[1] = (__nv_bfloat16*)a->out;              // X' = out + out_op
+        gi.xlo_out = (__nv_bfloat16*)a->out_op;
     }
     // unit lists of the two-CTA kernel (split tiles included, so the building
     // blocks exercise the partial-sum path too)

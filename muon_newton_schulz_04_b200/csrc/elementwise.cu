@@ -57,6 +57,30 @@ __device__ __forceinline__ float direction(float g, float* bptr, float mu, int n
     return nesterov ? fmaf(mu, bn, g) : bn;
 }
 
+// hi = bf16(x), lo = bf16(x - hi), for two values, packed as bf16x2 words
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+__device__ __forceinline__ void store_x0(const EwSeg& sg, size_t xo, float u, int bf16_operand) {
+    if (bf16_operand) {
+        const __nv_bfloat16 h = __float2bfloat16_rn(u);
+        sg.xhi0[xo] = h;
+        sg.xlo0[xo] = __float2bfloat16_rn(u - __bfloat162float(h));
+    } else {
+        sg.xf0[xo] = u;
+    }
+}
+
+// Element i (index into the oriented m x ldn iterate) of the final X.
+__device__ __forceinline__ float load_o(const EwSeg& sg, size_t i) {
+    return sg.o_hi ? __bfloat162float(sg.o_hi[i]) + __bfloat162float(sg.o_lo[i]) : sg.o_src[i];
+}
+
 __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* __restrict__ segs, int nseg,
                                                                   double* __restrict__ partials, float mu,
                                                                   int nesterov, int bf16_operand,
@@ -70,7 +94,7 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* 
     const EwSeg sg = segs[si];
     const int lb = blockIdx.x - sg.blk_begin;
     double acc = 0.0;
-    __nv_bfloat16* xb = reinterpret_cast<__nv_bfloat16*>(sg.xb0);
+    // bf16 path: X0 = hi + lo (hi = bf16(u), lo = bf16(u - hi)); fp32 debug path: X0 in fp32
 
     if (!sg.transposed) {
         const size_t total = (size_t)sg.rows * sg.cols;
@@ -104,16 +128,16 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* 
                 }
                 bp[0] = make_float4(b[0], b[1], b[2], b[3]);
                 bp[1] = make_float4(b[4], b[5], b[6], b[7]);
-                float4* xp = reinterpret_cast<float4*>(sg.xf0 + e);
-                xp[0] = make_float4(u[0], u[1], u[2], u[3]);
-                xp[1] = make_float4(u[4], u[5], u[6], u[7]);
                 if (bf16_operand) {
-                    uint4 w;
-                    __nv_bfloat162 h0 = __floats2bfloat162_rn(u[0], u[1]), h1 = __floats2bfloat162_rn(u[2], u[3]);
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(u[4], u[5]), h3 = __floats2bfloat162_rn(u[6], u[7]);
-                    w.x = *reinterpret_cast<uint32_t*>(&h0); w.y = *reinterpret_cast<uint32_t*>(&h1);
-                    w.z = *reinterpret_cast<uint32_t*>(&h2); w.w = *reinterpret_cast<uint32_t*>(&h3);
-                    *reinterpret_cast<uint4*>(xb + e) = w;
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) split_bf16x2(u[2 * i], u[2 * i + 1], hw[i], lw[i]);
+                    *reinterpret_cast<uint4*>(sg.xhi0 + e) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(sg.xlo0 + e) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                } else {
+                    float4* xp = reinterpret_cast<float4*>(sg.xf0 + e);
+                    xp[0] = make_float4(u[0], u[1], u[2], u[3]);
+                    xp[1] = make_float4(u[4], u[5], u[6], u[7]);
                 }
             }
         } else {
@@ -121,9 +145,7 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* 
                 const size_t r = e / (size_t)sg.cols, c = e - r * (size_t)sg.cols;
                 const float u = direction(load_g(sg.g, e, sg.g_bf16), sg.b ? sg.b + e : nullptr, mu, nesterov);
                 acc += (double)u * (double)u;
-                const size_t xo = r * (size_t)sg.ldn + c;
-                sg.xf0[xo] = u;
-                if (bf16_operand) xb[xo] = __float2bfloat16_rn(u);
+                store_x0(sg, r * (size_t)sg.ldn + c, u, bf16_operand);
             }
         }
     } else {
@@ -149,9 +171,7 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* 
             const int j = j0 + jj, i = i0 + tx;
             if (j < sg.cols && i < sg.rows) {
                 const float u = tile[tx][jj];
-                const size_t xo = (size_t)j * sg.ldn + i;
-                sg.xf0[xo] = u;
-                if (bf16_operand) xb[xo] = __float2bfloat16_rn(u);
+                store_x0(sg, (size_t)j * sg.ldn + i, u, bf16_operand);
             }
         }
     }
@@ -193,8 +213,21 @@ __device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay
         const size_t e1 = min(total, e0 + EW_FLAT_ELEMS);
         if (sg.vec) {
             for (size_t e = e0 + (size_t)threadIdx.x * 8; e < e1; e += (size_t)EW_THREADS * 8) {
-                const float4* op = reinterpret_cast<const float4*>(sg.o_src + e);
-                float4 o0 = op[0], o1 = op[1];
+                float4 o0, o1;
+                if (sg.o_hi) {
+                    const uint4 h = *reinterpret_cast<const uint4*>(sg.o_hi + e);
+                    const uint4 l = *reinterpret_cast<const uint4*>(sg.o_lo + e);
+                    auto f = [](uint32_t a, uint32_t b, bool hi_half) {
+                        return hi_half ? __uint_as_float(a & 0xFFFF0000u) + __uint_as_float(b & 0xFFFF0000u)
+                                       : __uint_as_float(a << 16) + __uint_as_float(b << 16);
+                    };
+                    o0 = make_float4(f(h.x, l.x, false), f(h.x, l.x, true), f(h.y, l.y, false), f(h.y, l.y, true));
+                    o1 = make_float4(f(h.z, l.z, false), f(h.z, l.z, true), f(h.w, l.w, false), f(h.w, l.w, true));
+                } else {
+                    const float4* op = reinterpret_cast<const float4*>(sg.o_src + e);
+                    o0 = op[0];
+                    o1 = op[1];
+                }
                 float4* wp = reinterpret_cast<float4*>(dst + e);
                 if (copy_out) {
                     o0.x *= os; o0.y *= os; o0.z *= os; o0.w *= os; o1.x *= os; o1.y *= os; o1.z *= os; o1.w *= os;
@@ -211,7 +244,7 @@ __device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay
         } else {
             for (size_t e = e0 + threadIdx.x; e < e1; e += EW_THREADS) {
                 const size_t r = e / (size_t)sg.cols, c = e - r * (size_t)sg.cols;
-                const float o = sg.o_src[r * (size_t)sg.ldn + c] * os;
+                const float o = load_o(sg, r * (size_t)sg.ldn + c) * os;
                 dst[e] = copy_out ? o : fmaf(-step, o, decay * dst[e]);
             }
         }
@@ -223,7 +256,7 @@ __device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay
 #pragma unroll 4
         for (int jj = ty; jj < EW_TILE; jj += 4) {
             const int j = j0 + jj, i = i0 + tx;
-            tile[jj][tx] = (j < sg.cols && i < sg.rows) ? sg.o_src[(size_t)j * sg.ldn + i] : 0.f;
+            tile[jj][tx] = (j < sg.cols && i < sg.rows) ? load_o(sg, (size_t)j * sg.ldn + i) : 0.f;
         }
         __syncthreads();
 #pragma unroll 4

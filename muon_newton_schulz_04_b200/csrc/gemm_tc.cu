@@ -253,46 +253,58 @@ __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const Gemm
             store_symmetric(gi.p + (size_t)mat * gi.m * gi.ldm, gi.m, gi.ldm, row, col0, val);
         } else {
             if (row < gi.m) {
+                // X = hi + lo in, X' = hi' + lo' out: hi' = bf16(X'), lo' = bf16(X' - hi')
                 const size_t off = (size_t)mat * gi.m * gi.ldn + (size_t)row * gi.ldn;
-                const float* xin = gi.xf_in + off;
-                float* xout = gi.xf_out + off;
-                __nv_bfloat16* xb = gi.xb[p.parity ^ 1] + off;
+                const __nv_bfloat16* hin = gi.xb[p.parity] + off;
+                const __nv_bfloat16* lin = gi.xlo_in + off;
+                __nv_bfloat16* hout = gi.xb[p.parity ^ 1] + off;
+                __nv_bfloat16* lout = gi.xlo_out + off;
                 if (col0 + 31 < gi.n) {
-                    const float4* src = reinterpret_cast<const float4*>(xin + col0);
+                    const uint4* hs = reinterpret_cast<const uint4*>(hin + col0);
+                    const uint4* ls = reinterpret_cast<const uint4*>(lin + col0);
+                    uint4 hw[4], lw[4];
 #pragma unroll
-                    for (int qq = 0; qq < 8; ++qq) {
-                        const float4 x = src[qq];
-                        val[4 * qq + 0] = alpha * __uint_as_float(v[4 * qq + 0]) + beta * x.x;
-                        val[4 * qq + 1] = alpha * __uint_as_float(v[4 * qq + 1]) + beta * x.y;
-                        val[4 * qq + 2] = alpha * __uint_as_float(v[4 * qq + 2]) + beta * x.z;
-                        val[4 * qq + 3] = alpha * __uint_as_float(v[4 * qq + 3]) + beta * x.w;
-                    }
-                    float4* dst = reinterpret_cast<float4*>(xout + col0);
+                    for (int qq = 0; qq < 4; ++qq) { hw[qq] = hs[qq]; lw[qq] = ls[qq]; }
 #pragma unroll
-                    for (int qq = 0; qq < 8; ++qq)
-                        dst[qq] = make_float4(val[4 * qq], val[4 * qq + 1], val[4 * qq + 2], val[4 * qq + 3]);
-                    if (p.write_op) {
-                        uint4* db = reinterpret_cast<uint4*>(xb + col0);
+                    for (int qq = 0; qq < 4; ++qq) {
+                        const uint32_t h4[4] = {hw[qq].x, hw[qq].y, hw[qq].z, hw[qq].w};
+                        const uint32_t l4[4] = {lw[qq].x, lw[qq].y, lw[qq].z, lw[qq].w};
+                        uint32_t ho[4], lo[4];
 #pragma unroll
-                        for (int qq = 0; qq < 4; ++qq) {
-                            uint4 w;
-                            w.x = pack_bf16x2(val[8 * qq + 0], val[8 * qq + 1]);
-                            w.y = pack_bf16x2(val[8 * qq + 2], val[8 * qq + 3]);
-                            w.z = pack_bf16x2(val[8 * qq + 4], val[8 * qq + 5]);
-                            w.w = pack_bf16x2(val[8 * qq + 6], val[8 * qq + 7]);
-                            db[qq] = w;
+                        for (int e = 0; e < 4; ++e) {
+                            const int j = 8 * qq + 2 * e;
+                            const float x0 = bf16_bits_lo(h4[e]) + bf16_bits_lo(l4[e]);
+                            const float x1 = bf16_bits_hi(h4[e]) + bf16_bits_hi(l4[e]);
+                            val[j] = alpha * __uint_as_float(v[j]) + beta * x0;
+                            val[j + 1] = alpha * __uint_as_float(v[j + 1]) + beta * x1;
+                            const __nv_bfloat162 hh = __floats2bfloat162_rn(val[j], val[j + 1]);
+                            const float2 hf = __bfloat1622float2(hh);
+                            const __nv_bfloat162 ll = __floats2bfloat162_rn(val[j] - hf.x, val[j + 1] - hf.y);
+                            ho[e] = *reinterpret_cast<const uint32_t*>(&hh);
+                            lo[e] = *reinterpret_cast<const uint32_t*>(&ll);
+                            // the stored pair is the result: the weight update uses exactly it
+                            const float2 lf = __bfloat1622float2(ll);
+                            val[j] = hf.x + lf.x;
+                            val[j + 1] = hf.y + lf.y;
                         }
+                        reinterpret_cast<uint4*>(hout + col0)[qq] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+                        reinterpret_cast<uint4*>(lout + col0)[qq] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
                     }
                 } else {
 #pragma unroll
                     for (int j = 0; j < 32; ++j) {
                         const int c = col0 + j;
-                        const float r = (c < gi.n) ? alpha * __uint_as_float(v[j]) + beta * xin[c] : 0.f;
-                        val[j] = r;
+                        float r = 0.f;
                         if (c < gi.n) {
-                            xout[c] = r;
-                            if (p.write_op) xb[c] = __float2bfloat16_rn(r);
+                            const float x = __bfloat162float(hin[c]) + __bfloat162float(lin[c]);
+                            r = alpha * __uint_as_float(v[j]) + beta * x;
+                            const __nv_bfloat16 hh = __float2bfloat16_rn(r);
+                            const __nv_bfloat16 ll = __float2bfloat16_rn(r - __bfloat162float(hh));
+                            hout[c] = hh;
+                            lout[c] = ll;
+                            r = __bfloat162float(hh) + __bfloat162float(ll);
                         }
+                        val[j] = r;
                     }
                 }
                 if (p.apply_mode != 0) apply_chunk(p, gi, mat, row, col0, val);

@@ -1,11 +1,12 @@
 // kernels.cuh -- device-side descriptors and kernel launchers of the Muon step.
 //
 // Layout in HBM (library-owned workspace, per group of same-shape matrices):
-//   xb[2]  bf16 [count][m][ldn]   operand copies of the iterate X (ping-pong)
-//   xf[.]  fp32 [count][m][ldn]   the iterate itself (1 buffer on the bf16 path,
-//                                 2 ping-pong buffers on the fp32 debug path)
+//   xb[2]  bf16 [count][m][ldn]   high part of the iterate, hi = bf16(X), which is
+//                                 also the tensor-core operand (ping-pong)
+//   xl     bf16 [count][m][ldn]   low part, lo = bf16(X - hi): X = hi + lo carries
+//                                 about 16 significant bits (updated in place)
 //   a, p   bf16 [count][m][ldm]   Gram matrix A = XX^T and P = bA + cA^2
-//                                 (fp32 on the debug path)
+// The fp32 debug path keeps X in two fp32 ping-pong buffers and A, P in fp32.
 // with m = min(rows, cols), n = max(rows, cols), ldm / ldn rounded up to 8
 // elements so that every row starts on a 16-byte boundary (a TMA requirement).
 // The caller's W, G, B stay where the caller put them.
@@ -32,9 +33,12 @@ struct EwSeg {
     const void* g;        // gradient (step) or input M (orthogonalize): rows x cols
     float* b;             // momentum buffer (nullptr: no momentum, U = G)
     float* w;             // weight (apply) or output O (copy-out)
-    float* xf0;           // fp32 iterate written by the momentum kernel (m x ldn)
-    void* xb0;            // bf16 operand copy written by the momentum kernel (nullptr on fp32 path)
-    const float* o_src;   // final fp32 iterate read by the apply kernel (m x ldn)
+    float* xf0;           // fp32 debug path: X0 written by the momentum kernel (m x ldn)
+    __nv_bfloat16* xhi0;  // bf16 path: X0 = hi + lo written by the momentum kernel
+    __nv_bfloat16* xlo0;
+    const float* o_src;   // fp32 debug path: final iterate read by the apply kernel
+    const __nv_bfloat16* o_hi;   // bf16 path: final iterate = o_hi + o_lo
+    const __nv_bfloat16* o_lo;
     int rows, cols;       // of W
     int ldn;              // row stride of the oriented iterate
     int transposed;       // rows > cols: X = U^T
@@ -59,9 +63,9 @@ struct GemmGroupInfo {
     int m, n, ldm, ldn;
     int count;
     int mat_base;                 // global index of this group's matrix 0
-    __nv_bfloat16* xb[2];
-    const float* xf_in;           // UPDATE: fp32 X read for the beta term
-    float* xf_out;                // UPDATE: fp32 X' written
+    __nv_bfloat16* xb[2];         // high parts of X (ping-pong; the GEMM operand)
+    const __nv_bfloat16* xlo_in;  // UPDATE: low part of X read for the beta term
+    __nv_bfloat16* xlo_out;       // UPDATE: low part of X' written (equal to xlo_in in a step)
     __nv_bfloat16* a;             // GRAM output / POLY input
     __nv_bfloat16* p;             // POLY output / UPDATE input (via map)
 };
@@ -74,7 +78,7 @@ struct GemmParams {
     int parity;                   // which xb holds the current iterate
     float alpha, beta;            // GRAM: alpha; POLY: alpha = c, beta = b; UPDATE: alpha = 1, beta = a
     const float* scale;           // per-matrix 1/(||U||+eps) on the first iteration, else nullptr
-    int write_op;                 // UPDATE: also write the bf16 operand copy of X'
+    int write_op;                 // unused (kept for the layout of the launch parameters)
     int* err;                     // device error word (bounded waits)
     // UPDATE of the last iteration only: 1 = also apply W <- decay*W - lr*s*O,
     // 2 = also copy O out to the caller (orthogonalisation), 0 = neither.
