@@ -245,12 +245,15 @@ int muon_plan_tile_n(void);
 muon_status muon_plan_tiles(const int* shapes, int n_groups, int phase, int* out, int cap, int* n_tiles);
 
 /* Work units of one launch of the two-CTA GEMM kernel built for `clusters`
- * two-CTA clusters: 10 ints per unit (cluster, group, matrix, tile_row, tile_col,
- * k_begin, k_end, kind, slot, nslots), k in 64-element blocks.  kind 0 = a whole
- * tile; 1 = the first K range of a split tile, which adds the partial sums of
- * slots [slot, slot + nslots); 2 = a later K range, which stores its partial sum
- * to `slot`.  Same conventions as muon_plan_tiles. */
-muon_status muon_plan_units(const int* shapes, int n_groups, int phase, int clusters, int* out, int cap,
+ * two-CTA clusters: 11 ints per unit (cluster, group, matrix, tile_row, tile_col,
+ * k_begin, k_end, kind, slot, nslots, n_half), k in 64-element blocks.
+ * split = 0 (the default schedule): whole tiles, the last partial round cut along
+ * N into 128-column halves when they fit one per cluster (n_half 1 / 2).
+ * split = 1: the K-blocks of the last partial round are divided over all clusters;
+ * kind 0 = a whole tile; 1 = the first K range of a split tile, which adds the
+ * partial sums of slots [slot, slot + nslots); 2 = a later K range, which stores
+ * its partial sum to `slot`.  Same conventions as muon_plan_tiles. */
+muon_status muon_plan_units(const int* shapes, int n_groups, int phase, int clusters, int split, int* out, int cap,
                             int* n_units);
 
 #ifdef __cplusplus

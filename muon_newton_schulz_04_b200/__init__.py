@@ -80,7 +80,8 @@ _SIGNATURES = {
                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float, ctypes.c_int,
                                                   ctypes.c_void_p, ctypes.c_void_p, ctypes.c_char_p, ctypes.c_int]),
     "muon_plan_units": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.c_int, ctypes.c_int,
-                                       ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.POINTER(ctypes.c_int)]),
+                                       ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.c_int,
+                                       ctypes.POINTER(ctypes.c_int)]),
     "muon_plan_tile_m": (ctypes.c_int, []),
     "muon_plan_tile_n": (ctypes.c_int, []),
     "muon_plan_tiles": (ctypes.c_int, [ctypes.POINTER(ctypes.c_int), ctypes.c_int, ctypes.c_int,
@@ -300,17 +301,17 @@ def plan_tiles(shapes, phase: int):
     return [tuple(out[4 * i: 4 * i + 4]) for i in range(n.value)]
 
 
-def plan_units(shapes, phase: int, clusters: int):
+def plan_units(shapes, phase: int, clusters: int, split: bool = False):
     """Work units of a two-CTA GEMM launch (host only): tuples (cluster, group, matrix,
-    tile_row, tile_col, k_begin, k_end, kind, slot, nslots)."""
+    tile_row, tile_col, k_begin, k_end, kind, slot, nslots, n_half)."""
     flat = (ctypes.c_int * (3 * len(shapes)))(*[int(v) for s in shapes for v in s])
     n = ctypes.c_int(0)
-    lib().muon_plan_units(flat, len(shapes), phase, clusters, None, 0, ctypes.byref(n))
-    out = (ctypes.c_int * (10 * max(n.value, 1)))()
-    st = lib().muon_plan_units(flat, len(shapes), phase, clusters, out, n.value, ctypes.byref(n))
+    lib().muon_plan_units(flat, len(shapes), phase, clusters, int(split), None, 0, ctypes.byref(n))
+    out = (ctypes.c_int * (11 * max(n.value, 1)))()
+    st = lib().muon_plan_units(flat, len(shapes), phase, clusters, int(split), out, n.value, ctypes.byref(n))
     if st != MUON_OK:
         raise MuonError(st, "muon_plan_units")
-    return [tuple(out[10 * i: 10 * i + 10]) for i in range(n.value)]
+    return [tuple(out[11 * i: 11 * i + 11]) for i in range(n.value)]
 
 
 def tile_shape():

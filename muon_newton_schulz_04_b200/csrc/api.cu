@@ -353,7 +353,7 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
                     const GroupDims& d = P.dims[t.group];
                     kb.push_back(((ph == 0 ? d.n : d.m) + TC_BK - 1) / TC_BK);
                 }
-                upl[ph] = build_units(*lists[ph], kb, h->max_clusters, tc_gemm_split_tiles() != 0);
+                upl[ph] = build_units(*lists[ph], kb, h->max_clusters, tc_gemm_split_tiles() != 0, true);
                 sk_slots = std::max(sk_slots, upl[ph].nslots);
             }
             P.unit_clusters = h->max_clusters;
@@ -449,7 +449,7 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
         for (int ph = 0; ph < 3 && h->pair; ++ph) {
             for (const Unit& u : upl[ph].units) {
                 uv[ph].push_back(make_int4(u.tile.group, u.tile.mat, u.tile.tile_row, u.tile.tile_col));
-                uv[ph].push_back(make_int4(u.k_begin, u.k_end, u.kind, u.slot | (u.nslots << 16)));
+                uv[ph].push_back(make_int4(u.k_begin, u.k_end, u.kind | (u.n_half << 8), u.slot | (u.nslots << 16)));
             }
             if (!uv[ph].empty())
                 CUDA_TRY(h, cudaMemcpyAsync(P.d_units[ph], uv[ph].data(), uv[ph].size() * sizeof(int4),
@@ -913,12 +913,12 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     if (h->pair) {
         std::vector<int> kb;
         for (size_t i = 0; i < tl.size(); ++i) kb.push_back(((phase == MUON_NS_GRAM ? n : m) + TC_BK - 1) / TC_BK);
-        up = build_units(tl, kb, h->max_clusters, tc_gemm_split_tiles() != 0);
+        up = build_units(tl, kb, h->max_clusters, tc_gemm_split_tiles() != 0, true);
     }
     std::vector<int4> uv;
     for (const Unit& u : up.units) {
         uv.push_back(make_int4(u.tile.group, u.tile.mat, u.tile.tile_row, u.tile.tile_col));
-        uv.push_back(make_int4(u.k_begin, u.k_end, u.kind, u.slot | (u.nslots << 16)));
+        uv.push_back(make_int4(u.k_begin, u.k_end, u.kind | (u.n_half << 8), u.slot | (u.nslots << 16)));
     }
     size_t off = 0;
     auto take = [&](size_t bytes) { size_t o = align_up(off, 256); off = o + align_up(bytes, 256); return o; };
@@ -1085,8 +1085,8 @@ muon_status muon_plan_tiles(const int* shapes, int n_groups, int phase, int* out
     return MUON_OK;
 }
 
-muon_status muon_plan_units(const int* shapes, int n_groups, int phase, int clusters, int* out, int cap,
-                            int* n_units) {
+muon_status muon_plan_units(const int* shapes, int n_groups, int phase, int clusters, int split, int* out,
+                            int cap, int* n_units) {
     if (!shapes || n_groups <= 0 || !n_units || phase < 0 || phase > 2 || clusters < 1) return MUON_ERR_INVALID;
     std::vector<GroupDims> dims;
     for (int g = 0; g < n_groups; ++g) {
@@ -1097,15 +1097,15 @@ muon_status muon_plan_units(const int* shapes, int n_groups, int phase, int clus
     std::vector<Tile> t = build_tiles(dims, phase, tc_gemm_tile_m(1), tc_gemm_tile_n(1));
     std::vector<int> kb;
     for (const Tile& x : t) kb.push_back(((phase == 0 ? dims[x.group].n : dims[x.group].m) + TC_BK - 1) / TC_BK);
-    UnitPlan up = build_units(t, kb, clusters, true);
+    UnitPlan up = build_units(t, kb, clusters, split != 0, split == 0);
     *n_units = (int)up.units.size();
     if (!out || cap < (int)up.units.size()) return MUON_ERR_INVALID;
     for (int c = 0; c < clusters; ++c) {
         for (int i = up.begin[c]; i < up.begin[c + 1]; ++i) {
             const Unit& u = up.units[i];
-            int* o = out + 10 * i;
+            int* o = out + 11 * i;
             o[0] = c; o[1] = u.tile.group; o[2] = u.tile.mat; o[3] = u.tile.tile_row; o[4] = u.tile.tile_col;
-            o[5] = u.k_begin; o[6] = u.k_end; o[7] = u.kind; o[8] = u.slot; o[9] = u.nslots;
+            o[5] = u.k_begin; o[6] = u.k_end; o[7] = u.kind; o[8] = u.slot; o[9] = u.nslots; o[10] = u.n_half;
         }
     }
     return MUON_OK;

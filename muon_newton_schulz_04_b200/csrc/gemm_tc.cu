@@ -188,7 +188,7 @@ __device__ __forceinline__ void apply_chunk(const GemmParams& p, const GemmGroup
 template <int MODE>
 __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const GemmGroupInfo& gi, int mat, int row,
                                                  int col_base, uint32_t tacc, int c_begin, int kind = 0,
-                                                 float* sk_row = nullptr, int nslots = 0) {
+                                                 float* sk_row = nullptr, int nslots = 0, int nchunks = 4) {
     float alpha = p.alpha, beta = p.beta;
     if (p.scale != nullptr) {
         const float s = p.scale[gi.mat_base + mat];
@@ -196,7 +196,7 @@ __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const Gemm
         if (MODE == MODE_UPDATE) { alpha = p.alpha * s; beta = p.beta * s; }
     }
 #pragma unroll 1
-    for (int chunk = 0; chunk < 4; ++chunk) {
+    for (int chunk = 0; chunk < nchunks; ++chunk) {
         const int c_local = c_begin + chunk * 32;
         uint32_t v[32];
         tmem_ld_32x32b_x32(tacc + (uint32_t)c_local, v);
@@ -541,8 +541,9 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
                 const int4 sk = p.units[2 * u + 1];
                 const void *mapA, *mapB;
                 operand_maps<MODE>(p, tile.x, mapA, mapB);
+                const int nh = sk.z >> 8;                              // 0: full tile, 1/2: column half
                 const int row0 = tile.z * S2_BM + (int)rank * 128;     // this CTA's rows of A
-                const int colh = tile.w * S2_BN + (int)rank * 128;     // this CTA's columns of B
+                const int colh = tile.w * S2_BN + (nh ? (nh - 1) * 128 + (int)rank * 64 : (int)rank * 128);
                 const int mat = tile.y;
                 for (int kb = sk.x; kb < sk.y; ++kb) {
                     if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, ERR_PRODUCER)) { ok = false; break; }
@@ -569,13 +570,15 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
         }
     } else if (warp == 1) {
         if (rank == 0 && elect_one()) {
-            constexpr uint32_t idesc = idesc_bf16_f32(S2_BM, S2_BN, MODE == MODE_UPDATE ? 1u : 0u);
+            constexpr uint32_t idesc_full = idesc_bf16_f32(S2_BM, S2_BN, MODE == MODE_UPDATE ? 1u : 0u);
+            constexpr uint32_t idesc_half = idesc_bf16_f32(S2_BM, S2_BN / 2, MODE == MODE_UPDATE ? 1u : 0u);
             uint32_t stage = 0, phase = 0;
             int local = 0;
             bool ok = true;
             const int u_end = p.unit_begin[cid + 1];
             for (int u = p.unit_begin[cid]; u < u_end && ok; ++u, ++local) {
                 const int4 sk = p.units[2 * u + 1];
+                const uint32_t idesc = (sk.z >> 8) ? idesc_half : idesc_full;
                 const uint32_t acc = local & 1;
                 const uint32_t acc_phase = (local >> 1) & 1;
                 if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.err, ERR_MMA_ACC)) { ok = false; break; }
@@ -618,7 +621,7 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
         for (int u = p.unit_begin[cid]; u < u_end; ++u, ++local) {
             const int4 tile = p.units[2 * u];
             const int4 sk = p.units[2 * u + 1];
-            const int kind = sk.z, slot = sk.w & 0xFFFF, nsl = sk.w >> 16;
+            const int kind = sk.z & 0xFF, nh = sk.z >> 8, slot = sk.w & 0xFFFF, nsl = sk.w >> 16;
             const GemmGroupInfo& gi = p.groups[tile.x];
             const uint32_t acc = local & 1;
             const uint32_t acc_phase = (local >> 1) & 1;
@@ -635,9 +638,10 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
             const int row = tile.z * S2_BM + (int)rank * 128 + row_local;
             float* sk_row = kind == 0 ? nullptr
                           : p.sk_partial + (size_t)slot * SK_SLOT_FLOATS + ((size_t)rank * 128 + row_local) * 256;
-            epilogue_segment<MODE>(p, gi, tile.y, row, tile.w * S2_BN,
-                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * 128, kind, sk_row,
-                                   nsl);
+            // a column half (nh = 1, 2) has 128 accumulator columns: 2 chunks per warp
+            epilogue_segment<MODE>(p, gi, tile.y, row, tile.w * S2_BN + (nh ? (nh - 1) * 128 : 0),
+                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * (nh ? 64 : 128), kind,
+                                   sk_row, nsl, nh ? 2 : 4);
             tc_fence_before();
             if (kind == 2) __threadfence();
             __syncwarp();

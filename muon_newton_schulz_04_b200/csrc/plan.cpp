@@ -52,14 +52,27 @@ std::vector<Tile> build_tiles(const std::vector<GroupDims>& groups, int phase, i
     return out;
 }
 
-UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kblocks, int clusters, bool split) {
+UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kblocks, int clusters, bool split,
+                     bool half_tail) {
     UnitPlan up;
     const int T = (int)tiles.size();
     const int C = clusters < 1 ? 1 : clusters;
-    const int R = split ? T % C : 0;
+    const int rem = T % C;
+    const bool halves = !split && half_tail && rem > 0 && T >= C && 2 * rem <= C;
+    const int R = (split || halves) ? rem : 0;
     const int D = T - R;
     std::vector<std::vector<Unit>> per(C);
-    for (int t = 0; t < D; ++t) per[t % C].push_back(Unit{tiles[t], 0, kblocks[t], 0, 0, 0});
+    for (int t = 0; t < D; ++t) per[t % C].push_back(Unit{tiles[t], 0, kblocks[t], 0, 0, 0, 0});
+    if (halves) {
+        for (int r = 0; r < R; ++r)
+            for (int h = 0; h < 2; ++h) per[2 * r + h].push_back(Unit{tiles[D + r], 0, kblocks[D + r], 0, 0, 0, 1 + h});
+        up.begin.push_back(0);
+        for (int c = 0; c < C; ++c) {
+            up.units.insert(up.units.end(), per[c].begin(), per[c].end());
+            up.begin.push_back((int)up.units.size());
+        }
+        return up;
+    }
     if (R > 0) {
         // flatten the remaining tiles' K-blocks and cut them into C ranges
         long long total = 0;
@@ -78,7 +91,7 @@ UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kbl
                 const int kb = (int)(a - start[r]), ke = (int)(e - start[r]);
                 tile_units[r].push_back(c);
                 tile_pos[r].push_back((int)sk[c].size());
-                sk[c].push_back(Unit{tiles[D + r], kb, ke, kb == 0 ? 1 : 2, 0, 0});
+                sk[c].push_back(Unit{tiles[D + r], kb, ke, kb == 0 ? 1 : 2, 0, 0, 0});
                 a = e;
                 ++r;
             }

@@ -39,7 +39,9 @@ std::vector<Tile> build_tiles(const std::vector<GroupDims>& groups, int phase, i
 // nearly equal ranges, one per cluster, so every cluster ends at about the same
 // time.  A cluster's range starts with at most one kind-2 unit, so a head unit only
 // waits for partials that their clusters produce before doing anything else.
-struct Unit { Tile tile; int k_begin, k_end, kind, slot, nslots; };
+//   n_half: 0 = all 256 columns of the tile; 1 / 2 = its first / second 128 columns
+//           (an independent output block with the full K range).
+struct Unit { Tile tile; int k_begin, k_end, kind, slot, nslots, n_half; };
 
 struct UnitPlan {
     std::vector<Unit> units;
@@ -47,7 +49,11 @@ struct UnitPlan {
     int nslots = 0;           // partial-sum slots used
 };
 
-UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kblocks, int clusters, bool split);
+// half_tail: when split is false and the R = T % C remaining tiles fit as 2R halves
+// on the C clusters (2R <= C), they are cut along N into two 128-column halves,
+// one per cluster, so the last round takes about half as long.
+UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kblocks, int clusters, bool split,
+                     bool half_tail = false);
 
 // 0 unless the environment variable MUON_GEMM_SPLIT is "1": split the K-blocks of
 // the last, partial round of tiles over all clusters (build_units).  Off by

@@ -164,19 +164,27 @@ def test_symmetric_tiles_skip_the_lower_triangle():
     assert sym < 0.56 * full
 
 
-@pytest.mark.parametrize("shapes,clusters", [([(4096, 4096, 1)], 74), ([(4096, 4096, 1)], 5), ([(256, 512, 1)], 74),
-                                             ([(768, 768, 4), (3072, 768, 1)], 74), ([(2048, 1408, 3)], 74),
-                                             ([(1024, 1536, 1)], 74), ([(1600, 1600, 2), (6400, 1600, 1)], 74)])
-@pytest.mark.parametrize("phase", [0, 1, 2])
-def test_units_cover_each_k_block_once_and_never_chain_waits(shapes, clusters, phase):
-    units = mb.plan_units(shapes, phase, clusters)
-    tiles = mb.plan_tiles(shapes, phase)
+UNIT_CASES = [([(4096, 4096, 1)], 74), ([(4096, 4096, 1)], 5), ([(256, 512, 1)], 74),
+              ([(768, 768, 4), (3072, 768, 1)], 74), ([(2048, 1408, 3)], 74),
+              ([(1024, 1536, 1)], 74), ([(1600, 1600, 2), (6400, 1600, 1)], 74)]
+
+
+def _kblocks(shapes, phase, tiles):
     dims = [(min(r, c), max(r, c)) for (r, c, _) in shapes]
-    kbl = {t: ((dims[t[0]][1] if phase == 0 else dims[t[0]][0]) + 63) // 64 for t in tiles}
+    return {t: ((dims[t[0]][1] if phase == 0 else dims[t[0]][0]) + 63) // 64 for t in tiles}
+
+
+@pytest.mark.parametrize("shapes,clusters", UNIT_CASES)
+@pytest.mark.parametrize("phase", [0, 1, 2])
+def test_split_units_cover_each_k_block_once_and_never_chain_waits(shapes, clusters, phase):
+    units = mb.plan_units(shapes, phase, clusters, split=True)
+    tiles = mb.plan_tiles(shapes, phase)
+    kbl = _kblocks(shapes, phase, tiles)
     seen = {t: [] for t in tiles}
     by_cluster = {}
     slots = {}
-    for (c, g, z, tr, tc, kb, ke, kind, slot, nsl) in units:
+    for (c, g, z, tr, tc, kb, ke, kind, slot, nsl, nh) in units:
+        assert nh == 0
         seen[(g, z, tr, tc)].append((kb, ke, kind, slot, nsl, c))
         by_cluster.setdefault(c, []).append(kind)
         if kind == 2:
@@ -201,6 +209,29 @@ def test_units_cover_each_k_block_once_and_never_chain_waits(shapes, clusters, p
         # partial, before any wait: producers never wait, so waits cannot chain
         assert all(k != 1 for k in kinds[:-1]) and kinds.count(2) <= 1
     assert set(c for (c, *_r) in units) <= set(range(clusters))
+
+
+@pytest.mark.parametrize("shapes,clusters", UNIT_CASES)
+@pytest.mark.parametrize("phase", [0, 1, 2])
+def test_default_units_cover_each_tile_once(shapes, clusters, phase):
+    units = mb.plan_units(shapes, phase, clusters, split=False)
+    tiles = mb.plan_tiles(shapes, phase)
+    kbl = _kblocks(shapes, phase, tiles)
+    seen = {t: [] for t in tiles}
+    load = {}
+    for (c, g, z, tr, tc, kb, ke, kind, slot, nsl, nh) in units:
+        assert kind == 0 and kb == 0 and ke == kbl[(g, z, tr, tc)]
+        seen[(g, z, tr, tc)].append((nh, c))
+        load[c] = load.get(c, 0) + (1.0 if nh == 0 else 0.5)
+    for t, parts in seen.items():
+        halves = sorted(nh for (nh, _c) in parts)
+        assert halves in ([0], [1, 2]), (t, parts)
+        if halves == [1, 2]:
+            assert parts[0][1] != parts[1][1]                                       # halves on two clusters
+    T = len(tiles)
+    assert max(load.values()) <= -(-T // clusters)                                  # never worse than whole tiles
+    if T >= clusters and 0 < 2 * (T % clusters) <= clusters:
+        assert max(load.values()) == T // clusters + 0.5                            # the tail round is halved
 
 
 def test_no_undefined_library_symbols():

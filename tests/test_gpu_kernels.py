@@ -41,7 +41,10 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
 
-SHAPES = [(128, 256, 1), (320, 776, 3), (384, 384, 2), (136, 1032, 1), (8, 64, 2), (520, 264, 1), (1024, 1536, 1)]
+# (2048, 2560): 80 update tiles on 74 clusters -> the tail round runs as 128-column halves;
+# (3328, 3328): 91 Gram / polynomial tiles -> the same for the symmetric products.
+SHAPES = [(128, 256, 1), (320, 776, 3), (384, 384, 2), (136, 1032, 1), (8, 64, 2), (520, 264, 1), (1024, 1536, 1),
+          (2048, 2560, 1), (3328, 3328, 1)]
 
 
 @pytest.mark.parametrize("m,n,count", SHAPES)
