@@ -7,10 +7,10 @@ links it, and it shares no code with the library.
 from .muon_oracle import (NS_COEFFS, NS_STEPS, DEFAULT_EPS, SCALE_NONE, SCALE_MATCH_RMS,
                           SCALE_CUSTOM, momentum_accumulate, nesterov_direction, orient,
                           frobenius_normalize, gram, poly_matrix, ns_update, ns_iteration,
-                          newton_schulz, shape_scale, apply_update, muon_step, muon_steps)
+                          newton_schulz, shape_scale, apply_update, muon_step, muon_steps, qk_clip)
 from .jacobi_svd import jacobi_svd
 
 __all__ = ["NS_COEFFS", "NS_STEPS", "DEFAULT_EPS", "SCALE_NONE", "SCALE_MATCH_RMS", "SCALE_CUSTOM",
            "momentum_accumulate", "nesterov_direction", "orient", "frobenius_normalize", "gram",
            "poly_matrix", "ns_update", "ns_iteration", "newton_schulz", "shape_scale",
-           "apply_update", "muon_step", "muon_steps", "jacobi_svd"]
+           "apply_update", "muon_step", "muon_steps", "qk_clip", "jacobi_svd"]

@@ -157,3 +157,22 @@ def muon_steps(W0: np.ndarray, grads: Sequence[np.ndarray], **hp) -> List[Dict[s
         W, B = res["W"], res["B"]
         out.append(res)
     return out
+
+
+def qk_clip(Wq: np.ndarray, Wk: np.ndarray, max_logits: Sequence[float], tau: float,
+            head_dim: int) -> Tuple[np.ndarray, np.ndarray]:
+    """QK-Clip of MuonClip (section "关键实验/定理", result 3: after the Muon step the
+    query and key projections of each attention head are rescaled according to that
+    head's maximum attention logit).  The page gives no formula.  Reading: with
+    gamma_h = min(1, tau / S_h) for the head's maximum logit S_h, the rows of head h
+    (rows h*head_dim .. (h+1)*head_dim - 1 of W_q and of W_k, PyTorch Linear layout)
+    are multiplied by sqrt(gamma_h), so every logit q.k of the head is multiplied
+    by gamma_h and the head's maximum logit becomes min(S_h, tau)."""
+    Wq = np.asarray(Wq, dtype=np.float64).copy()
+    Wk = np.asarray(Wk, dtype=np.float64).copy()
+    for h, s in enumerate(max_logits):
+        gamma = min(1.0, tau / float(s)) if s > 0 else 1.0
+        f = math.sqrt(gamma)
+        Wq[h * head_dim:(h + 1) * head_dim, :] *= f
+        Wk[h * head_dim:(h + 1) * head_dim, :] *= f
+    return Wq, Wk

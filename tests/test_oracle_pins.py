@@ -306,3 +306,45 @@ def test_pins_catch_planted_iteration_mistakes(fn, shape, monkeypatch):
 def test_pins_catch_planted_step_mistakes(name, fn, monkeypatch):
     monkeypatch.setattr(mo, name, fn)
     assert _chain_error() > 1e-6
+
+
+# ----------------------------------------------------------------------------- QK-Clip
+
+def _head_max_logits(Wq, Wk, Xin, head_dim):
+    """Per-head maximum of q.k over all query/key token pairs of the input batch."""
+    q = Xin @ Wq.T
+    k = Xin @ Wk.T
+    out = []
+    for h in range(Wq.shape[0] // head_dim):
+        sl = slice(h * head_dim, (h + 1) * head_dim)
+        out.append(float(np.max(q[:, sl] @ k[:, sl].T)))
+    return out
+
+
+def test_qk_clip_caps_each_head_at_tau():
+    rng = np.random.default_rng(71)
+    heads, hd, d = 4, 8, 32
+    Wq = rng.standard_normal((heads * hd, d))
+    Wk = rng.standard_normal((heads * hd, d))
+    Xin = rng.standard_normal((10, d))
+    S = _head_max_logits(Wq, Wk, Xin, hd)
+    tau = float(np.median(S))
+    Wq2, Wk2 = oracle.qk_clip(Wq, Wk, S, tau, hd)
+    S2 = _head_max_logits(Wq2, Wk2, Xin, hd)
+    for s, s2 in zip(S, S2):
+        assert abs(s2 - min(s, tau)) <= 1e-9 * abs(s)
+    # heads at or below tau are bit-for-bit untouched
+    for h, s in enumerate(S):
+        if s <= tau:
+            assert np.array_equal(Wq2[h * hd:(h + 1) * hd], Wq[h * hd:(h + 1) * hd])
+
+
+def test_qk_clip_pin_catches_unsplit_scale(monkeypatch):
+    """Scaling only W_q by gamma (not sqrt(gamma) on both) also caps the logits, but the
+    pages' reading splits it: check the factor on each side."""
+    rng = np.random.default_rng(72)
+    Wq = rng.standard_normal((8, 4))
+    Wk = rng.standard_normal((8, 4))
+    Wq2, Wk2 = oracle.qk_clip(Wq, Wk, [4.0, 1.0], 1.0, 4)
+    assert np.allclose(Wq2[:4], 0.5 * Wq[:4]) and np.allclose(Wk2[:4], 0.5 * Wk[:4])
+    assert np.array_equal(Wq2[4:], Wq[4:]) and np.array_equal(Wk2[4:], Wk[4:])
