@@ -170,6 +170,17 @@ typedef struct {
 
 muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* args, void* stream);
 
+/* QK-Clip of MuonClip ("关键实验/定理" result 3: after the Muon step, each attention
+ * head's query and key projections are rescaled according to the head's maximum
+ * logit; the page gives no formula).  With gamma_h = min(1, tau / max_logits[h]),
+ * the rows of head h -- rows h*head_dim .. (h+1)*head_dim - 1 -- of Wq and of Wk
+ * are multiplied by sqrt(gamma_h), so every logit of the head scales by gamma_h.
+ * Wq, Wk: fp32 (n_heads*head_dim) x cols, row-major, device, updated in place
+ * (Wk may be NULL); max_logits: n_heads floats, device, produced by the caller's
+ * attention; tau > 0. */
+muon_status muon_qk_clip(muon_handle* h, float* Wq, float* Wk, const float* max_logits, int n_heads, int head_dim,
+                         int cols, float tau, void* stream);
+
 /* Waits for the handle's work on `stream`, then reports a kernel that gave up a
  * bounded wait (MUON_ERR_DEVICE_TIMEOUT, flag cleared) or an asynchronous CUDA
  * error (MUON_ERR_CUDA). */

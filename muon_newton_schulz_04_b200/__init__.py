@@ -66,6 +66,8 @@ _SIGNATURES = {
     "muon_step_host": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_Group), ctypes.c_int, ctypes.c_void_p]),
     "muon_orthogonalize": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_OrthoGroup), ctypes.c_int, ctypes.c_void_p]),
     "muon_ns_phase_run": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_PhaseArgs), ctypes.c_void_p]),
+    "muon_qk_clip": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                                    ctypes.c_int, ctypes.c_int, ctypes.c_float, ctypes.c_void_p]),
     "muon_sync": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "muon_last_norms": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_float), ctypes.c_int,
                                        ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]),
@@ -233,6 +235,17 @@ class Muon:
         args = _PhaseArgs(phase, precision, m, n, count, alpha, beta, p(x_op), p(a_in), p(x_master), p(out), p(out_op))
         self._check(lib().muon_ns_phase_run(self._h, ctypes.byref(args), ctypes.c_void_p(_stream(stream))),
                     "muon_ns_phase_run")
+
+    def qk_clip(self, Wq, Wk, max_logits, head_dim: int, tau: float, stream=None):
+        """MuonClip's QK-Clip: rows of head h of Wq and Wk times sqrt(min(1, tau / max_logits[h]))."""
+        n_heads = max_logits.numel()
+        rows, cols = Wq.shape
+        if rows != n_heads * head_dim or (Wk is not None and tuple(Wk.shape) != (rows, cols)):
+            raise ValueError("Wq / Wk must be (n_heads * head_dim) x cols")
+        self._check(lib().muon_qk_clip(self._h, ctypes.c_void_p(Wq.data_ptr()),
+                                       None if Wk is None else ctypes.c_void_p(Wk.data_ptr()),
+                                       ctypes.c_void_p(max_logits.data_ptr()), n_heads, head_dim, cols, float(tau),
+                                       ctypes.c_void_p(_stream(stream))), "muon_qk_clip")
 
     def sync(self, stream=None):
         self._check(lib().muon_sync(self._h, ctypes.c_void_p(_stream(stream))), "muon_sync")

@@ -964,6 +964,22 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     return MUON_OK;
 }
 
+muon_status muon_qk_clip(muon_handle* h, float* Wq, float* Wk, const float* max_logits, int n_heads, int head_dim,
+                         int cols, float tau, void* stream) {
+    if (!h) return MUON_ERR_INVALID;
+    if (!Wq || !max_logits) return fail(h, MUON_ERR_INVALID, "Wq and max_logits are required");
+    if (n_heads <= 0 || head_dim <= 0 || cols <= 0) return fail(h, MUON_ERR_INVALID, "sizes must be > 0");
+    if ((long long)n_heads * head_dim * cols > (1ll << 31) - 1) return fail(h, MUON_ERR_INVALID, "matrix too large");
+    if (!(finite(tau) && tau > 0.f)) return fail(h, MUON_ERR_INVALID, "tau must be finite and > 0");
+    if (!aligned(Wq, 4) || (Wk && !aligned(Wk, 4)) || !aligned(max_logits, 4))
+        return fail(h, MUON_ERR_INVALID, "misaligned pointer");
+    DeviceGuard dg(h->device);
+    h->last_error.clear();
+    CUDA_TRY(h, launch_qk_clip(Wq, Wk, max_logits, n_heads, head_dim, cols, tau, h->num_sms,
+                               static_cast<cudaStream_t>(stream)));
+    return MUON_OK;
+}
+
 muon_status muon_sync(muon_handle* h, void* stream) {
     if (!h) return MUON_ERR_INVALID;
     DeviceGuard dg(h->device);

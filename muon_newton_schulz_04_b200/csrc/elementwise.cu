@@ -16,8 +16,17 @@
 // matrices take a flat path (8 elements per thread per access, 16/32-byte
 // vectors); tall matrices go through a 64x64 shared-memory transpose so that
 // both the row-major reads and the transposed writes stay coalesced.
+#include <algorithm>
+
 #include "kernels.cuh"
 #include "ptx.cuh"
+
+#ifndef EW_GROUPS_IN_FLIGHT
+#define EW_GROUPS_IN_FLIGHT 2
+#endif
+#ifndef EW_MIN_BLOCKS
+#define EW_MIN_BLOCKS 4
+#endif
 
 namespace muon {
 namespace {
@@ -81,7 +90,7 @@ __device__ __forceinline__ float load_o(const EwSeg& sg, size_t i) {
     return sg.o_hi ? __bfloat162float(sg.o_hi[i]) + __bfloat162float(sg.o_lo[i]) : sg.o_src[i];
 }
 
-__global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* __restrict__ segs, int nseg,
+__global__ void __launch_bounds__(EW_THREADS, EW_MIN_BLOCKS) momentum_norm_kernel(const EwSeg* __restrict__ segs, int nseg,
                                                                   double* __restrict__ partials, float mu,
                                                                   int nesterov, int bf16_operand,
                                                                   int* __restrict__ counters, float eps,
@@ -101,31 +110,59 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* 
         const size_t e0 = (size_t)lb * EW_FLAT_ELEMS;
         const size_t e1 = min(total, e0 + EW_FLAT_ELEMS);
         if (sg.vec && sg.b != nullptr) {
-            // rows are dense and 8-aligned: the oriented X has the same flat index
-            for (size_t e = e0 + (size_t)threadIdx.x * 8; e < e1; e += (size_t)EW_THREADS * 8) {
+            // rows are dense and 8-aligned: the oriented X has the same flat index.
+            // All loads of the thread's (up to) 4 groups of 8 elements are issued
+            // before any arithmetic: 12 (bf16 G) or 16 (fp32 G) 16-byte loads per
+            // thread in flight.  bf16 G stays packed until it is used.
+            constexpr int GROUPS = EW_FLAT_ELEMS / (EW_THREADS * 8);
+            constexpr int GB = EW_GROUPS_IN_FLIGHT;
+#pragma unroll 1
+            for (int k0 = 0; k0 < GROUPS; k0 += GB) {
+            uint4 graw[GB][2];
+            float4 braw[GB][2];
+#pragma unroll
+            for (int kk = 0; kk < GB; ++kk) {
+                const int k = k0 + kk;
+                const size_t e = e0 + ((size_t)k * EW_THREADS + threadIdx.x) * 8;
+                if (e >= e1) continue;
+                if (sg.g_bf16) {
+                    graw[kk][0] = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(sg.g) + e);
+                } else {
+                    graw[kk][0] = *reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(sg.g) + e);
+                    graw[kk][1] = *reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(sg.g) + e + 4);
+                }
+                const float4* bp = reinterpret_cast<const float4*>(sg.b + e);
+                braw[kk][0] = bp[0];
+                braw[kk][1] = bp[1];
+            }
+#pragma unroll
+            for (int kk = 0; kk < GB; ++kk) {
+                const int k = k0 + kk;
+                const size_t e = e0 + ((size_t)k * EW_THREADS + threadIdx.x) * 8;
+                if (e >= e1) continue;
                 float g[8], b[8], u[8];
                 if (sg.g_bf16) {
-                    const uint4 raw = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(sg.g) + e);
-                    const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+                    const uint32_t w[4] = {graw[kk][0].x, graw[kk][0].y, graw[kk][0].z, graw[kk][0].w};
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         g[2 * i] = __uint_as_float(w[i] << 16);
                         g[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
                     }
                 } else {
-                    const float4 a0 = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(sg.g) + e);
-                    const float4 a1 = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(sg.g) + e + 4);
-                    g[0] = a0.x; g[1] = a0.y; g[2] = a0.z; g[3] = a0.w; g[4] = a1.x; g[5] = a1.y; g[6] = a1.z; g[7] = a1.w;
+                    const uint32_t w[8] = {graw[kk][0].x, graw[kk][0].y, graw[kk][0].z, graw[kk][0].w,
+                                           graw[kk][1].x, graw[kk][1].y, graw[kk][1].z, graw[kk][1].w};
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) g[i] = __uint_as_float(w[i]);
                 }
-                float4* bp = reinterpret_cast<float4*>(sg.b + e);
-                const float4 b0 = bp[0], b1 = bp[1];
-                b[0] = b0.x; b[1] = b0.y; b[2] = b0.z; b[3] = b0.w; b[4] = b1.x; b[5] = b1.y; b[6] = b1.z; b[7] = b1.w;
+                b[0] = braw[kk][0].x; b[1] = braw[kk][0].y; b[2] = braw[kk][0].z; b[3] = braw[kk][0].w;
+                b[4] = braw[kk][1].x; b[5] = braw[kk][1].y; b[6] = braw[kk][1].z; b[7] = braw[kk][1].w;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     b[i] = fmaf(mu, b[i], g[i]);
                     u[i] = nesterov ? fmaf(mu, b[i], g[i]) : b[i];
                     acc += (double)u[i] * (double)u[i];
                 }
+                float4* bp = reinterpret_cast<float4*>(sg.b + e);
                 bp[0] = make_float4(b[0], b[1], b[2], b[3]);
                 bp[1] = make_float4(b[4], b[5], b[6], b[7]);
                 if (bf16_operand) {
@@ -140,6 +177,7 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* 
                     xp[1] = make_float4(u[4], u[5], u[6], u[7]);
                 }
             }
+            }
         } else {
             for (size_t e = e0 + threadIdx.x; e < e1; e += EW_THREADS) {
                 const size_t r = e / (size_t)sg.cols, c = e - r * (size_t)sg.cols;
@@ -152,26 +190,102 @@ __global__ void __launch_bounds__(EW_THREADS) momentum_norm_kernel(const EwSeg* 
         // tall matrix: X = U^T.  Tile of U rows [i0, i0+64) x cols [j0, j0+64).
         const int tiles_c = (sg.cols + EW_TILE - 1) / EW_TILE;
         const int i0 = (lb / tiles_c) * EW_TILE, j0 = (lb % tiles_c) * EW_TILE;
-        const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;     // 64 x 4
-#pragma unroll 4
-        for (int ii = ty; ii < EW_TILE; ii += 4) {
-            const int i = i0 + ii, j = j0 + tx;
-            float u = 0.f;
-            if (i < sg.rows && j < sg.cols) {
+        if (sg.vec && sg.b != nullptr) {
+            // 16 x 16 threads, each on 4 consecutive columns of 4 rows (r, r+16, r+32,
+            // r+48): every G and B load of the thread is issued before any arithmetic.
+            // cols % 8 == 0, so a 4-column group is either wholly inside or outside.
+            const int c4 = threadIdx.x & 15, r = threadIdx.x >> 4;
+            const int j = j0 + 4 * c4;
+            constexpr int RSTEPS = EW_TILE / 16;
+            uint4 graw[RSTEPS];
+            float4 braw[RSTEPS];
+#pragma unroll
+            for (int k = 0; k < RSTEPS; ++k) {
+                const int i = i0 + r + 16 * k;
+                if (i >= sg.rows || j >= sg.cols) continue;
                 const size_t e = (size_t)i * sg.cols + j;
-                u = direction(load_g(sg.g, e, sg.g_bf16), sg.b ? sg.b + e : nullptr, mu, nesterov);
-                acc += (double)u * (double)u;
+                if (sg.g_bf16) {
+                    const uint2 v = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(sg.g) + e);
+                    graw[k] = make_uint4(v.x, v.y, 0u, 0u);
+                } else {
+                    graw[k] = *reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(sg.g) + e);
+                }
+                braw[k] = *reinterpret_cast<const float4*>(sg.b + e);
             }
-            tile[ii][tx] = u;
-        }
-        __syncthreads();
-        // write X[j][i] = U[i][j]: consecutive threads take consecutive i
+#pragma unroll
+            for (int k = 0; k < RSTEPS; ++k) {
+                const int i = i0 + r + 16 * k;
+                float u[4] = {0.f, 0.f, 0.f, 0.f};
+                if (i < sg.rows && j < sg.cols) {
+                    float g[4];
+                    if (sg.g_bf16) {
+                        g[0] = __uint_as_float(graw[k].x << 16);
+                        g[1] = __uint_as_float(graw[k].x & 0xFFFF0000u);
+                        g[2] = __uint_as_float(graw[k].y << 16);
+                        g[3] = __uint_as_float(graw[k].y & 0xFFFF0000u);
+                    } else {
+                        g[0] = __uint_as_float(graw[k].x); g[1] = __uint_as_float(graw[k].y);
+                        g[2] = __uint_as_float(graw[k].z); g[3] = __uint_as_float(graw[k].w);
+                    }
+                    float b[4] = {braw[k].x, braw[k].y, braw[k].z, braw[k].w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        b[q] = fmaf(mu, b[q], g[q]);
+                        u[q] = nesterov ? fmaf(mu, b[q], g[q]) : b[q];
+                        acc += (double)u[q] * (double)u[q];
+                    }
+                    *reinterpret_cast<float4*>(sg.b + (size_t)i * sg.cols + j) = make_float4(b[0], b[1], b[2], b[3]);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) tile[r + 16 * k][4 * c4 + q] = u[q];
+            }
+            __syncthreads();
+            // X[jx][i0 + 4*c4 .. +3] = U[i][jx]: 4 consecutive elements of an X row per thread
+            const int ix = i0 + 4 * c4;
+#pragma unroll
+            for (int k = 0; k < RSTEPS; ++k) {
+                const int jj = r + 16 * k, jx = j0 + jj;
+                if (jx >= sg.cols || ix >= sg.rows) continue;
+                float u[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) u[q] = tile[4 * c4 + q][jj];
+                const size_t xo = (size_t)jx * sg.ldn + ix;
+                if (ix + 3 < sg.rows) {
+                    if (bf16_operand) {
+                        uint32_t hw[2], lw[2];
+                        split_bf16x2(u[0], u[1], hw[0], lw[0]);
+                        split_bf16x2(u[2], u[3], hw[1], lw[1]);
+                        *reinterpret_cast<uint2*>(sg.xhi0 + xo) = make_uint2(hw[0], hw[1]);
+                        *reinterpret_cast<uint2*>(sg.xlo0 + xo) = make_uint2(lw[0], lw[1]);
+                    } else {
+                        *reinterpret_cast<float4*>(sg.xf0 + xo) = make_float4(u[0], u[1], u[2], u[3]);
+                    }
+                } else {
+                    for (int q = 0; ix + q < sg.rows; ++q) store_x0(sg, xo + q, u[q], bf16_operand);
+                }
+            }
+        } else {
+            const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;     // 64 x 4
 #pragma unroll 4
-        for (int jj = ty; jj < EW_TILE; jj += 4) {
-            const int j = j0 + jj, i = i0 + tx;
-            if (j < sg.cols && i < sg.rows) {
-                const float u = tile[tx][jj];
-                store_x0(sg, (size_t)j * sg.ldn + i, u, bf16_operand);
+            for (int ii = ty; ii < EW_TILE; ii += 4) {
+                const int i = i0 + ii, j = j0 + tx;
+                float u = 0.f;
+                if (i < sg.rows && j < sg.cols) {
+                    const size_t e = (size_t)i * sg.cols + j;
+                    u = direction(load_g(sg.g, e, sg.g_bf16), sg.b ? sg.b + e : nullptr, mu, nesterov);
+                    acc += (double)u * (double)u;
+                }
+                tile[ii][tx] = u;
+            }
+            __syncthreads();
+            // write X[j][i] = U[i][j]: consecutive threads take consecutive i
+#pragma unroll 4
+            for (int jj = ty; jj < EW_TILE; jj += 4) {
+                const int j = j0 + jj, i = i0 + tx;
+                if (j < sg.cols && i < sg.rows) {
+                    const float u = tile[tx][jj];
+                    store_x0(sg, (size_t)j * sg.ldn + i, u, bf16_operand);
+                }
             }
         }
     }
@@ -305,6 +419,54 @@ cudaError_t launch_apply(const EwSeg* segs, int nseg, int nblocks, float decay, 
 cudaError_t launch_copy_out_one(const EwSeg& seg, float* dst, const float* o_scale, cudaStream_t s) {
     if (seg.apply_count <= 0) return cudaSuccess;
     return launch_pdl(copy_out_one_kernel, dim3(seg.apply_count), dim3(EW_THREADS), 0, s, seg, dst, o_scale);
+}
+
+}  // namespace muon
+
+// ---------------------------------------------------------------- QK-Clip
+// After the Muon step, MuonClip rescales each attention head's rows of the query
+// and key projections by sqrt(gamma_h), gamma_h = min(1, tau / S_h) for the head's
+// maximum logit S_h (the Kimi K2 result of the Muon synthesis note), so every logit
+// of the head scales by gamma_h.  One launch covers W_q and W_k; blockIdx.y picks
+// the matrix.  Rows are grouped by head: head = row / head_dim.
+namespace muon {
+namespace {
+
+__global__ void __launch_bounds__(EW_THREADS) qk_clip_kernel(float* __restrict__ wq, float* __restrict__ wk,
+                                                            const float* __restrict__ max_logits, int head_dim,
+                                                            int cols, size_t total, float tau, int vec) {
+    pdl_trigger();
+    pdl_wait();
+    float* w = blockIdx.y == 0 ? wq : wk;
+    if (w == nullptr) return;
+    const size_t stride = (size_t)gridDim.x * EW_THREADS * (vec ? 4 : 1);
+    for (size_t e = ((size_t)blockIdx.x * EW_THREADS + threadIdx.x) * (vec ? 4 : 1); e < total; e += stride) {
+        const int head = (int)((e / (size_t)cols) / (size_t)head_dim);
+        const float s = max_logits[head];
+        const float f = s > tau ? sqrtf(tau / s) : 1.0f;
+        if (f == 1.0f) continue;
+        if (vec) {
+            float4 x = *reinterpret_cast<float4*>(w + e);
+            x.x *= f; x.y *= f; x.z *= f; x.w *= f;
+            *reinterpret_cast<float4*>(w + e) = x;
+        } else {
+            w[e] *= f;
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_qk_clip(float* wq, float* wk, const float* max_logits, int n_heads, int head_dim, int cols,
+                           float tau, int num_sms, cudaStream_t s) {
+    const size_t total = (size_t)n_heads * head_dim * cols;
+    if (total == 0) return cudaSuccess;
+    const int vec = (cols % 4 == 0) && (reinterpret_cast<uintptr_t>(wq) % 16 == 0) &&
+                    (wk == nullptr || reinterpret_cast<uintptr_t>(wk) % 16 == 0);
+    const size_t work = vec ? total / 4 : total;
+    const int blocks = (int)std::min<size_t>((work + EW_THREADS - 1) / EW_THREADS, (size_t)num_sms * 8);
+    return launch_pdl(qk_clip_kernel, dim3(blocks, 2), dim3(EW_THREADS), 0, s, wq, wk, max_logits, head_dim, cols,
+                      total, tau, vec);
 }
 
 }  // namespace muon

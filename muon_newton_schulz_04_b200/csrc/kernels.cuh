@@ -134,6 +134,10 @@ cudaError_t launch_momentum_norm(const EwSeg* segs, int nseg, int nblocks, doubl
 cudaError_t launch_apply(const EwSeg* segs, int nseg, int nblocks, float decay, float lr,
                          const float* o_scale, int copy_out, cudaStream_t s);
 cudaError_t launch_copy_out_one(const EwSeg& seg, float* dst, const float* o_scale, cudaStream_t s);
+// QK-Clip: rows of head h of W_q and W_k (n_heads * head_dim rows, `cols` columns)
+// times sqrt(min(1, tau / max_logits[h])).  wk may be nullptr.
+cudaError_t launch_qk_clip(float* wq, float* wk, const float* max_logits, int n_heads, int head_dim, int cols,
+                           float tau, int num_sms, cudaStream_t s);
 
 // Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger in
 // ptx.cuh): the kernel may start while the previous kernel of the stream drains and

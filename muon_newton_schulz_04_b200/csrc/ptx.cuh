@@ -288,6 +288,16 @@ namespace muon {
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// L2 prefetch of `bytes` contiguous bytes (16-byte aligned address, size a multiple
+// of 16): the bulk-copy engine pulls the range into L2 without occupying registers.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* gptr, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(gptr), "r"(bytes) : "memory");
+}
+// L2 prefetch of the cache line holding `gptr`.
+__device__ __forceinline__ void prefetch_l2_line(const void* gptr) {
+    asm volatile("prefetch.global.L2 [%0];" :: "l"(gptr));
+}
+
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 }  // namespace muon

@@ -38,16 +38,20 @@ def _step_one(shapes, cfg, grads, weights, dtype=torch.float32):
     return out
 
 
-ODD = [(37, 1000), (1000, 37), (1, 64), (64, 1), (1, 1), (129, 257), (300, 129), (8, 8)]
+ODD = [(37, 1000), (1000, 37), (1, 64), (64, 1), (1, 1), (129, 257), (300, 129), (8, 8),
+       (1001, 72), (130, 8)]          # tall with 8-aligned columns: vector transpose, ragged rows
 
 
-@pytest.mark.parametrize("precision", [mb.PREC_BF16, mb.PREC_FP32_DEBUG])
-def test_odd_shapes_one_call(precision):
+@pytest.mark.parametrize("precision,gdtype", [(mb.PREC_BF16, torch.float32), (mb.PREC_FP32_DEBUG, torch.float32),
+                                              (mb.PREC_BF16, torch.bfloat16)])
+def test_odd_shapes_one_call(precision, gdtype):
     rng = np.random.default_rng(5)
     G = [rng.standard_normal(s).astype(np.float32) for s in ODD]
+    # the oracle sees the gradient the kernel reads: bf16-rounded when G is bf16
+    G = [torch.from_numpy(g).to(gdtype).float().numpy() for g in G]
     W0 = [0.02 * rng.standard_normal(s) for s in ODD]
     cfg = mb.config(precision=precision, weight_decay=0.1)
-    W, B, O = _step_one(ODD, cfg, G, W0)
+    W, B, O = _step_one(ODD, cfg, G, W0, dtype=gdtype)
     for i, s in enumerate(ODD):
         res = oracle.muon_step(W0[i].astype(np.float32).astype(np.float64), G[i].astype(np.float64),
                                np.zeros(s), lr=0.02, momentum=0.95, nesterov=True, weight_decay=0.1, eps=1e-7)
