@@ -44,11 +44,17 @@ constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
 constexpr int ACC_COLS = 256;                 // one accumulator: 128 lanes x 256 fp32 columns
 constexpr int TMEM_COLS = 2 * ACC_COLS;       // two accumulators
 
+// per epilogue warp: a 32 x 32 fp32 chunk for the UPDATE epilogue's re-layout,
+// rows padded to 33 words so that both access patterns are free of bank conflicts
+constexpr int STAGE_LD = 33;
+constexpr int STAGE_FLOATS = 32 * STAGE_LD;
+constexpr int STAGE_BYTES = NUM_EPI_WARPS * STAGE_FLOATS * 4;
+
 // one-CTA kernel
 constexpr int S1_BM = 128, S1_BN = 256, S1_STAGES = 4;
 constexpr int S1_A = S1_BM * BK * 2;          // 16 KiB
 constexpr int S1_B = S1_BN * BK * 2;          // 32 KiB
-constexpr int S1_SMEM = 1024 + S1_STAGES * (S1_A + S1_B) + 256;
+constexpr int S1_SMEM = 1024 + S1_STAGES * (S1_A + S1_B) + 256 + STAGE_BYTES;
 
 // two-CTA kernel (per CTA)
 #ifndef MUON_S2_STAGES
@@ -57,7 +63,8 @@ constexpr int S1_SMEM = 1024 + S1_STAGES * (S1_A + S1_B) + 256;
 constexpr int S2_BM = 256, S2_BN = 256, S2_STAGES = MUON_S2_STAGES;
 constexpr int S2_A = 128 * BK * 2;            // 16 KiB: this CTA's 128 rows of A
 constexpr int S2_B = 128 * BK * 2;            // 16 KiB: this CTA's 128 columns of B
-constexpr int S2_SMEM = 1024 + S2_STAGES * (S2_A + S2_B) + 256;
+constexpr int S2_SMEM = 1024 + S2_STAGES * (S2_A + S2_B) + 256 + STAGE_BYTES;
+static_assert(S1_SMEM <= 232448 && S2_SMEM <= 232448, "dynamic shared memory above the 227 KiB limit");
 
 // error codes written to the device error word when a bounded wait gives up
 constexpr int ERR_PRODUCER = 0x101, ERR_MMA_SLOT = 0x102, ERR_MMA_ACC = 0x103, ERR_EPILOGUE = 0x104,
@@ -176,6 +183,153 @@ __device__ __forceinline__ void apply_chunk(const GemmParams& p, const GemmGroup
     }
 }
 
+// UPDATE epilogue operands of one thread, pulled into L2 while the tile's MMAs run:
+// the thread's `ncols` columns from `col_start` of its row of X = hi + lo and, when
+// the weight update is fused (apply_mode 1), the matching elements of W.  Every
+// range stays inside its buffer: X rows end at ldn (a multiple of 8 elements),
+// W is touched only inside its rows x cols.
+__device__ __forceinline__ void prefetch_update_operands(const GemmParams& p, const GemmGroupInfo& gi, int mat,
+                                                         int row, int col_start, int ncols) {
+    if (row >= gi.m || col_start >= gi.n) return;
+    const int nc = min(ncols, gi.ldn - col_start);
+    const size_t off = (size_t)mat * gi.m * gi.ldn + (size_t)row * gi.ldn + col_start;
+    prefetch_l2_bulk(gi.xb[p.parity] + off, (uint32_t)nc * 2u);
+    prefetch_l2_bulk(gi.xlo_in + off, (uint32_t)nc * 2u);
+    if (p.apply_mode != 1) return;
+    const EwSeg& sg = p.segs[gi.mat_base + mat];
+    const int ncw = min(ncols, gi.n - col_start);
+    if (!sg.transposed) {
+        const float* wr = sg.w + (size_t)row * sg.cols + col_start;
+        if (sg.vec) {
+            prefetch_l2_bulk(wr, (uint32_t)ncw * 4u);
+        } else {
+            for (int c = 0; c < ncw; c += 32) prefetch_l2_line(wr + c);
+        }
+    } else {
+        // W[c][row]: the warp's 32 consecutive rows are one 128-byte run of W's row c;
+        // lane l takes W rows col_start + l, col_start + l + 32, ...
+        const int lane = (int)(threadIdx.x & 31u);
+        const int row0 = row - lane;
+        for (int c = lane; c < ncw; c += 32) prefetch_l2_line(sg.w + (size_t)(col_start + c) * sg.cols + row0);
+    }
+}
+
+// Weight update (apply_mode 1) or copy-out (apply_mode 2) of 8 finished values
+// O[r][c..c+7] of a matrix that was not transposed (W has the layout of O).
+__device__ __forceinline__ void apply_run8(const GemmParams& p, const EwSeg& sg, int n, int r, int c,
+                                           const float (&val)[8]) {
+    float* wr = sg.w + (size_t)r * sg.cols + c;
+    const float step = p.lr * sg.update_scale;
+    const bool copy = p.apply_mode == 2;
+    if (sg.vec && c + 7 < n) {
+        float4* w4 = reinterpret_cast<float4*>(wr);
+#pragma unroll
+        for (int qq = 0; qq < 2; ++qq) {
+            float4 o = make_float4(val[4 * qq], val[4 * qq + 1], val[4 * qq + 2], val[4 * qq + 3]);
+            if (!copy) {
+                const float4 x = w4[qq];
+                o.x = fmaf(-step, o.x, p.decay * x.x);
+                o.y = fmaf(-step, o.y, p.decay * x.y);
+                o.z = fmaf(-step, o.z, p.decay * x.z);
+                o.w = fmaf(-step, o.w, p.decay * x.w);
+            }
+            w4[qq] = o;
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (c + k < n) wr[k] = copy ? val[k] : fmaf(-step, val[k], p.decay * wr[k]);
+    }
+}
+
+// UPDATE epilogue of one 32 x 32 chunk: X' = alpha * acc + beta * (hi + lo), stored
+// as the pair hi' = bf16(X'), lo' = bf16(X' - hi').  The accumulator arrives one row
+// per lane (tcgen05.ld 32x32b); it goes through the warp's shared buffer so that lane
+// l works on rows l/4 + 8i (i = 0..3), columns 8(l%4) .. 8(l%4)+7 of the chunk.  Each
+// 16-byte access of the warp then covers 8 rows x 64 contiguous bytes, a quarter of
+// the cache lines that the row-per-lane layout touches.  hw / lw: this lane's hi and
+// lo words in that layout, loaded by the caller (valid where the 8 columns are inside
+// the matrix).
+__device__ __forceinline__ void update_chunk(const GemmParams& p, const GemmGroupInfo& gi, int mat, int row,
+                                             int col0, float alpha, float beta, const uint32_t (&v)[32],
+                                             const uint4 (&hw)[4], const uint4 (&lw)[4], float* stage) {
+    const int lane = (int)(threadIdx.x & 31u);
+    const int row_w = row - lane;
+    const int lr = lane >> 2, lc = (lane & 3) * 8;
+    __syncwarp();                                   // the previous chunk's reads are done
+#pragma unroll
+    for (int j = 0; j < 32; ++j) stage[lane * STAGE_LD + j] = __uint_as_float(v[j]);
+    __syncwarp();
+    const EwSeg* sg = p.apply_mode != 0 ? &p.segs[gi.mat_base + mat] : nullptr;
+    const bool apply_t = sg != nullptr && sg->transposed;
+    float res[4][8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = row_w + lr + 8 * i, c = col0 + lc;
+        float acc8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            acc8[k] = stage[(lr + 8 * i) * STAGE_LD + lc + k];
+            res[i][k] = 0.f;
+        }
+        if (r >= gi.m) continue;
+        const size_t o = (size_t)mat * gi.m * gi.ldn + (size_t)r * gi.ldn + c;
+        __nv_bfloat16* hout = gi.xb[p.parity ^ 1] + o;
+        __nv_bfloat16* lout = gi.xlo_out + o;
+        if (c + 7 < gi.n) {
+            const uint32_t h4[4] = {hw[i].x, hw[i].y, hw[i].z, hw[i].w};
+            const uint32_t l4[4] = {lw[i].x, lw[i].y, lw[i].z, lw[i].w};
+            uint32_t ho[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float x0 = bf16_bits_lo(h4[e]) + bf16_bits_lo(l4[e]);
+                const float x1 = bf16_bits_hi(h4[e]) + bf16_bits_hi(l4[e]);
+                const float y0 = alpha * acc8[2 * e] + beta * x0;
+                const float y1 = alpha * acc8[2 * e + 1] + beta * x1;
+                const __nv_bfloat162 hh = __floats2bfloat162_rn(y0, y1);
+                const float2 hf = __bfloat1622float2(hh);
+                const __nv_bfloat162 ll = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
+                ho[e] = *reinterpret_cast<const uint32_t*>(&hh);
+                lo[e] = *reinterpret_cast<const uint32_t*>(&ll);
+                // the stored pair is the result: the weight update uses exactly it
+                const float2 lf = __bfloat1622float2(ll);
+                res[i][2 * e] = hf.x + lf.x;
+                res[i][2 * e + 1] = hf.y + lf.y;
+            }
+            *reinterpret_cast<uint4*>(hout) = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+            *reinterpret_cast<uint4*>(lout) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        } else {
+            const __nv_bfloat16* hin = gi.xb[p.parity] + o;
+            const __nv_bfloat16* lin = gi.xlo_in + o;
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                if (c + k >= gi.n) continue;
+                const float y = alpha * acc8[k] + beta * (__bfloat162float(hin[k]) + __bfloat162float(lin[k]));
+                const __nv_bfloat16 hh = __float2bfloat16_rn(y);
+                const __nv_bfloat16 ll = __float2bfloat16_rn(y - __bfloat162float(hh));
+                hout[k] = hh;
+                lout[k] = ll;
+                res[i][k] = __bfloat162float(hh) + __bfloat162float(ll);
+            }
+        }
+        if (sg != nullptr && !apply_t) apply_run8(p, *sg, gi.n, r, c, res[i]);
+    }
+    if (apply_t) {
+        // W[c][r] of a transposed matrix: back to one row per lane, where the warp's
+        // lanes are 32 consecutive elements of one row of W
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < 8; ++k) stage[(lr + 8 * i) * STAGE_LD + lc + k] = res[i][k];
+        __syncwarp();
+        float val[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) val[j] = stage[lane * STAGE_LD + j];
+        if (row < gi.m) apply_chunk(p, gi, mat, row, col0, val);
+    }
+}
+
 // Epilogue of one accumulator row segment: 4 chunks of 32 columns starting at
 // column `c_begin` of the accumulator whose TMEM address (lane quarter included)
 // is `tacc`.  `row` is the global output row of this thread, `col_base` the
@@ -187,8 +341,9 @@ __device__ __forceinline__ void apply_chunk(const GemmParams& p, const GemmGroup
 // usual epilogue; kind 0 is a whole tile.
 template <int MODE>
 __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const GemmGroupInfo& gi, int mat, int row,
-                                                 int col_base, uint32_t tacc, int c_begin, int kind = 0,
-                                                 float* sk_row = nullptr, int nslots = 0, int nchunks = 4) {
+                                                 int col_base, uint32_t tacc, int c_begin, float* stage,
+                                                 int kind = 0, float* sk_row = nullptr, int nslots = 0,
+                                                 int nchunks = 4) {
     float alpha = p.alpha, beta = p.beta;
     if (p.scale != nullptr) {
         const float s = p.scale[gi.mat_base + mat];
@@ -198,6 +353,24 @@ __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const Gemm
 #pragma unroll 1
     for (int chunk = 0; chunk < nchunks; ++chunk) {
         const int c_local = c_begin + chunk * 32;
+        const int col0 = col_base + c_local;
+        // UPDATE works in the coalesced layout (see update_chunk); the iterate's loads
+        // go out before the accumulator read so that their latency overlaps it.
+        const int lane = (int)(threadIdx.x & 31u);
+        const int row_w = row - lane;                  // first row of this warp's slice
+        const int lr = lane >> 2, lc = (lane & 3) * 8;
+        uint4 hw[4], lw[4];
+        if (MODE == MODE_UPDATE && kind != 2) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = row_w + lr + 8 * i, c = col0 + lc;
+                if (r < gi.m && c + 7 < gi.n) {
+                    const size_t o = (size_t)mat * gi.m * gi.ldn + (size_t)r * gi.ldn + c;
+                    hw[i] = *reinterpret_cast<const uint4*>(gi.xb[p.parity] + o);
+                    lw[i] = *reinterpret_cast<const uint4*>(gi.xlo_in + o);
+                }
+            }
+        }
         uint32_t v[32];
         tmem_ld_32x32b_x32(tacc + (uint32_t)c_local, v);
         tmem_ld_wait();
@@ -222,7 +395,6 @@ __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const Gemm
                 }
             }
         }
-        const int col0 = col_base + c_local;
         float val[32];
         if (MODE == MODE_GRAM) {
 #pragma unroll
@@ -252,63 +424,7 @@ __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const Gemm
             }
             store_symmetric(gi.p + (size_t)mat * gi.m * gi.ldm, gi.m, gi.ldm, row, col0, val);
         } else {
-            if (row < gi.m) {
-                // X = hi + lo in, X' = hi' + lo' out: hi' = bf16(X'), lo' = bf16(X' - hi')
-                const size_t off = (size_t)mat * gi.m * gi.ldn + (size_t)row * gi.ldn;
-                const __nv_bfloat16* hin = gi.xb[p.parity] + off;
-                const __nv_bfloat16* lin = gi.xlo_in + off;
-                __nv_bfloat16* hout = gi.xb[p.parity ^ 1] + off;
-                __nv_bfloat16* lout = gi.xlo_out + off;
-                if (col0 + 31 < gi.n) {
-                    const uint4* hs = reinterpret_cast<const uint4*>(hin + col0);
-                    const uint4* ls = reinterpret_cast<const uint4*>(lin + col0);
-                    uint4 hw[4], lw[4];
-#pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) { hw[qq] = hs[qq]; lw[qq] = ls[qq]; }
-#pragma unroll
-                    for (int qq = 0; qq < 4; ++qq) {
-                        const uint32_t h4[4] = {hw[qq].x, hw[qq].y, hw[qq].z, hw[qq].w};
-                        const uint32_t l4[4] = {lw[qq].x, lw[qq].y, lw[qq].z, lw[qq].w};
-                        uint32_t ho[4], lo[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int j = 8 * qq + 2 * e;
-                            const float x0 = bf16_bits_lo(h4[e]) + bf16_bits_lo(l4[e]);
-                            const float x1 = bf16_bits_hi(h4[e]) + bf16_bits_hi(l4[e]);
-                            val[j] = alpha * __uint_as_float(v[j]) + beta * x0;
-                            val[j + 1] = alpha * __uint_as_float(v[j + 1]) + beta * x1;
-                            const __nv_bfloat162 hh = __floats2bfloat162_rn(val[j], val[j + 1]);
-                            const float2 hf = __bfloat1622float2(hh);
-                            const __nv_bfloat162 ll = __floats2bfloat162_rn(val[j] - hf.x, val[j + 1] - hf.y);
-                            ho[e] = *reinterpret_cast<const uint32_t*>(&hh);
-                            lo[e] = *reinterpret_cast<const uint32_t*>(&ll);
-                            // the stored pair is the result: the weight update uses exactly it
-                            const float2 lf = __bfloat1622float2(ll);
-                            val[j] = hf.x + lf.x;
-                            val[j + 1] = hf.y + lf.y;
-                        }
-                        reinterpret_cast<uint4*>(hout + col0)[qq] = make_uint4(ho[0], ho[1], ho[2], ho[3]);
-                        reinterpret_cast<uint4*>(lout + col0)[qq] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                    }
-                } else {
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int c = col0 + j;
-                        float r = 0.f;
-                        if (c < gi.n) {
-                            const float x = __bfloat162float(hin[c]) + __bfloat162float(lin[c]);
-                            r = alpha * __uint_as_float(v[j]) + beta * x;
-                            const __nv_bfloat16 hh = __float2bfloat16_rn(r);
-                            const __nv_bfloat16 ll = __float2bfloat16_rn(r - __bfloat162float(hh));
-                            hout[c] = hh;
-                            lout[c] = ll;
-                            r = __bfloat162float(hh) + __bfloat162float(ll);
-                        }
-                        val[j] = r;
-                    }
-                }
-                if (p.apply_mode != 0) apply_chunk(p, gi, mat, row, col0, val);
-            }
+            update_chunk(p, gi, mat, row, col0, alpha, beta, v, hw, lw, stage);
         }
     }
 }
@@ -459,18 +575,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid
     } else {
         const uint32_t q = warp & 3u;
         const uint32_t half = (warp - 2) >> 2;
+        float* stage = reinterpret_cast<float*>(smem + S1_STAGES * (S1_A + S1_B) + 256) + (warp - 2) * STAGE_FLOATS;
         int local = 0;
         for (int t = blockIdx.x; t < p.ntiles; t += gridDim.x, ++local) {
             const int4 tile = p.tiles[t];
             const GemmGroupInfo& gi = p.groups[tile.x];
             const uint32_t acc = local & 1;
             const uint32_t acc_phase = (local >> 1) & 1;
+            const int row = tile.z * S1_BM + (int)(q * 32 + lane);
+            if (MODE == MODE_UPDATE)
+                prefetch_update_operands(p, gi, tile.y, row, tile.w * S1_BN + (int)half * 128, 128);
             bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, ERR_EPILOGUE);
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const int row = tile.z * S1_BM + (int)(q * 32 + lane);
             epilogue_segment<MODE>(p, gi, tile.y, row, tile.w * S1_BN,
-                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * 128);
+                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * 128, stage);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tempty[acc]);
@@ -616,6 +735,7 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
     } else {
         const uint32_t q = warp & 3u;
         const uint32_t half = (warp - 2) >> 2;
+        float* stage = reinterpret_cast<float*>(smem + S2_STAGES * (S2_A + S2_B) + 256) + (warp - 2) * STAGE_FLOATS;
         int local = 0;
         const int u_end = p.unit_begin[cid + 1];
         for (int u = p.unit_begin[cid]; u < u_end; ++u, ++local) {
@@ -625,6 +745,12 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
             const GemmGroupInfo& gi = p.groups[tile.x];
             const uint32_t acc = local & 1;
             const uint32_t acc_phase = (local >> 1) & 1;
+            const int row_local = (int)(q * 32 + lane);
+            const int row = tile.z * S2_BM + (int)rank * 128 + row_local;
+            if (MODE == MODE_UPDATE && kind != 2)
+                prefetch_update_operands(p, gi, tile.y, row,
+                                         tile.w * S2_BN + (nh ? (nh - 1) * 128 + (int)half * 64 : (int)half * 128),
+                                         nh ? 64 : 128);
             bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, ERR_EPILOGUE);
             if (kind == 1 && lane == 0) {
                 // the later parts of this split tile, produced first by other clusters
@@ -634,14 +760,12 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
             if (!__all_sync(0xffffffffu, ok)) break;
             tc_fence_after();
-            const int row_local = (int)(q * 32 + lane);
-            const int row = tile.z * S2_BM + (int)rank * 128 + row_local;
             float* sk_row = kind == 0 ? nullptr
                           : p.sk_partial + (size_t)slot * SK_SLOT_FLOATS + ((size_t)rank * 128 + row_local) * 256;
             // a column half (nh = 1, 2) has 128 accumulator columns: 2 chunks per warp
             epilogue_segment<MODE>(p, gi, tile.y, row, tile.w * S2_BN + (nh ? (nh - 1) * 128 : 0),
-                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * (nh ? 64 : 128), kind,
-                                   sk_row, nsl, nh ? 2 : 4);
+                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * (nh ? 64 : 128), stage,
+                                   kind, sk_row, nsl, nh ? 2 : 4);
             tc_fence_before();
             if (kind == 2) __threadfence();
             __syncwarp();
