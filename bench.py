@@ -163,7 +163,7 @@ def update_gemm_flops(w: wl.Workload):
 # has no counters until it is captured again.
 UPDATE_TRAFFIC = {
     # (source hash, workload key, variant) -> bytes per launch
-    ("a0483919b093a66c", "square4096", "pair"): 141.596672e6,     # profiles/ns_gemm_update_square4096.md
+    ("cd720dba274579e3", "square4096", "pair"): 160.373e6,     # profiles/ns_gemm_update_square4096.md
 }
 
 
