@@ -104,39 +104,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_bits_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_bits_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Stores one 32-column chunk of one output row of a symmetric output (GRAM, POLY).
-// Element (row, c) is stored directly when c >= row and mirrored to (c, row) when
-// c > row, so every element of the m x m output is written exactly once.
-__device__ __forceinline__ void store_symmetric(__nv_bfloat16* __restrict__ out, int m, int ldm,
-                                                int row, int col0, const float (&val)[32]) {
-    if (row >= m) return;
-    if (col0 >= row && col0 + 31 < m) {
-        uint4* dst = reinterpret_cast<uint4*>(out + (size_t)row * ldm + col0);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            uint4 w;
-            w.x = pack_bf16x2(val[8 * q + 0], val[8 * q + 1]);
-            w.y = pack_bf16x2(val[8 * q + 2], val[8 * q + 3]);
-            w.z = pack_bf16x2(val[8 * q + 4], val[8 * q + 5]);
-            w.w = pack_bf16x2(val[8 * q + 6], val[8 * q + 7]);
-            dst[q] = w;
-        }
-    } else {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int c = col0 + j;
-            if (c >= row && c < m) out[(size_t)row * ldm + c] = __float2bfloat16_rn(val[j]);
-        }
-    }
-    // mirror: lanes hold consecutive rows, so each store instruction of the warp
-    // writes 32 consecutive elements of row c.
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-        const int c = col0 + j;
-        if (c > row && c < m) out[(size_t)c * ldm + row] = __float2bfloat16_rn(val[j]);
-    }
-}
-
 // Update of the weight (apply_mode 1: W <- decay*W - lr*s*O, eq. 3 with decoupled
 // decay and the per-shape scale) or copy-out of O (apply_mode 2) for the 32
 // finished values O[row][col0..col0+31] of the oriented result.  A matrix that was
@@ -242,6 +209,16 @@ __device__ __forceinline__ void apply_run8(const GemmParams& p, const EwSeg& sg,
     }
 }
 
+// Writes the warp's accumulator chunk (one row per lane, as tcgen05.ld 32x32b
+// delivers it) into its shared buffer.
+__device__ __forceinline__ void stage_chunk(const uint32_t (&v)[32], float* stage) {
+    const int lane = (int)(threadIdx.x & 31u);
+    __syncwarp();                                   // the previous chunk's reads are done
+#pragma unroll
+    for (int j = 0; j < 32; ++j) stage[lane * STAGE_LD + j] = __uint_as_float(v[j]);
+    __syncwarp();
+}
+
 // UPDATE epilogue of one 32 x 32 chunk: X' = alpha * acc + beta * (hi + lo), stored
 // as the pair hi' = bf16(X'), lo' = bf16(X' - hi').  The accumulator arrives one row
 // per lane (tcgen05.ld 32x32b); it goes through the warp's shared buffer so that lane
@@ -256,10 +233,7 @@ __device__ __forceinline__ void update_chunk(const GemmParams& p, const GemmGrou
     const int lane = (int)(threadIdx.x & 31u);
     const int row_w = row - lane;
     const int lr = lane >> 2, lc = (lane & 3) * 8;
-    __syncwarp();                                   // the previous chunk's reads are done
-#pragma unroll
-    for (int j = 0; j < 32; ++j) stage[lane * STAGE_LD + j] = __uint_as_float(v[j]);
-    __syncwarp();
+    stage_chunk(v, stage);
     const EwSeg* sg = p.apply_mode != 0 ? &p.segs[gi.mat_base + mat] : nullptr;
     const bool apply_t = sg != nullptr && sg->transposed;
     float res[4][8];
@@ -330,6 +304,79 @@ __device__ __forceinline__ void update_chunk(const GemmParams& p, const GemmGrou
     }
 }
 
+// GRAM / POLY epilogue of one 32 x 32 chunk of a symmetric m x m output (only
+// tiles with tile column >= tile row run): y = alpha * acc, plus beta * A for the
+// polynomial.  Element (r, c) is stored at (r, c) when c >= r and mirrored to
+// (c, r) when c > r, so every element of the output is written exactly once.  The
+// chunk goes through the warp's shared buffer: the direct stores use the layout of
+// update_chunk (lane l: rows l/4 + 8i, 8 columns from 8(l%4)), the mirrored ones its
+// transpose (lane l: output row col0 + l/4 + 8i, 8 columns from row_w + 8(l%4)), so
+// each 16-byte store instruction of the warp covers 8 rows x 64 contiguous bytes.
+// aw: this lane's words of A in the first layout (polynomial only; valid where the 8
+// columns are inside the matrix).
+template <int MODE>
+__device__ __forceinline__ void sym_chunk(__nv_bfloat16* __restrict__ out, const __nv_bfloat16* A, int m, int ldm,
+                                          int row, int col0, float alpha, float beta, const uint32_t (&v)[32],
+                                          const uint4 (&aw)[4], float* stage) {
+    const int lane = (int)(threadIdx.x & 31u);
+    const int row_w = row - lane, lr = lane >> 2, lc = (lane & 3) * 8;
+    if (col0 + 31 < row_w) return;              // every element below the diagonal: nothing to store
+    stage_chunk(v, stage);
+    const bool above = col0 >= row_w + 32;      // every element has c > r
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int r = row_w + lr + 8 * i, c = col0 + lc;
+        float* slot = stage + (lr + 8 * i) * STAGE_LD + lc;
+        float y[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) y[k] = alpha * slot[k];
+        if (MODE == MODE_POLY) {
+            if (r < m && c + 7 < m) {
+                const uint32_t w4[4] = {aw[i].x, aw[i].y, aw[i].z, aw[i].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    y[2 * e] += beta * bf16_bits_lo(w4[e]);
+                    y[2 * e + 1] += beta * bf16_bits_hi(w4[e]);
+                }
+            } else {
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                    if (r < m && c + k < m) y[k] += beta * __bfloat162float(A[(size_t)r * ldm + c + k]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) slot[k] = y[k];
+        if (r >= m) continue;
+        if (above && c + 7 < m) {
+            *reinterpret_cast<uint4*>(out + (size_t)r * ldm + c) =
+                make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                           pack_bf16x2(y[6], y[7]));
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (c + k >= r && c + k < m) out[(size_t)r * ldm + c + k] = __float2bfloat16_rn(y[k]);
+        }
+    }
+    __syncwarp();                               // every lane's values are in the buffer
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int cc = col0 + lr + 8 * i, rr = row_w + lc;   // output row cc holds column cc's mirror
+        if (cc >= m) continue;
+        float y[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) y[k] = stage[(lc + k) * STAGE_LD + lr + 8 * i];
+        if (above && rr + 7 < m) {
+            *reinterpret_cast<uint4*>(out + (size_t)cc * ldm + rr) =
+                make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                           pack_bf16x2(y[6], y[7]));
+        } else {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                if (cc > rr + k && rr + k < m) out[(size_t)cc * ldm + rr + k] = __float2bfloat16_rn(y[k]);
+        }
+    }
+}
+
 // Epilogue of one accumulator row segment: 4 chunks of 32 columns starting at
 // column `c_begin` of the accumulator whose TMEM address (lane quarter included)
 // is `tacc`.  `row` is the global output row of this thread, `col_base` the
@@ -360,6 +407,15 @@ __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const Gemm
         const int row_w = row - lane;                  // first row of this warp's slice
         const int lr = lane >> 2, lc = (lane & 3) * 8;
         uint4 hw[4], lw[4];
+        if (MODE == MODE_POLY && kind != 2) {
+            // the polynomial's b A term, in the same layout
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = row_w + lr + 8 * i, c = col0 + lc;
+                if (r < gi.m && c + 7 < gi.m)
+                    hw[i] = *reinterpret_cast<const uint4*>(gi.a + (size_t)mat * gi.m * gi.ldm + (size_t)r * gi.ldm + c);
+            }
+        }
         if (MODE == MODE_UPDATE && kind != 2) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -395,34 +451,12 @@ __device__ __forceinline__ void epilogue_segment(const GemmParams& p, const Gemm
                 }
             }
         }
-        float val[32];
         if (MODE == MODE_GRAM) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) val[j] = alpha * __uint_as_float(v[j]);
-            store_symmetric(gi.a + (size_t)mat * gi.m * gi.ldm, gi.m, gi.ldm, row, col0, val);
+            sym_chunk<MODE_GRAM>(gi.a + (size_t)mat * gi.m * gi.ldm, nullptr, gi.m, gi.ldm, row, col0, alpha, beta,
+                                 v, hw, stage);
         } else if (MODE == MODE_POLY) {
-            const __nv_bfloat16* A = gi.a + (size_t)mat * gi.m * gi.ldm;
-            if (row < gi.m && col0 + 31 < gi.m) {
-                const uint4* src = reinterpret_cast<const uint4*>(A + (size_t)row * gi.ldm + col0);
-#pragma unroll
-                for (int qq = 0; qq < 4; ++qq) {
-                    const uint4 w = src[qq];
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        val[8 * qq + 2 * e] = alpha * __uint_as_float(v[8 * qq + 2 * e]) + beta * bf16_bits_lo(ws[e]);
-                        val[8 * qq + 2 * e + 1] = alpha * __uint_as_float(v[8 * qq + 2 * e + 1]) + beta * bf16_bits_hi(ws[e]);
-                    }
-                }
-            } else {
-#pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int c = col0 + j;
-                    const float av = (row < gi.m && c < gi.m) ? __bfloat162float(A[(size_t)row * gi.ldm + c]) : 0.f;
-                    val[j] = alpha * __uint_as_float(v[j]) + beta * av;
-                }
-            }
-            store_symmetric(gi.p + (size_t)mat * gi.m * gi.ldm, gi.m, gi.ldm, row, col0, val);
+            sym_chunk<MODE_POLY>(gi.p + (size_t)mat * gi.m * gi.ldm, gi.a + (size_t)mat * gi.m * gi.ldm, gi.m, gi.ldm,
+                                 row, col0, alpha, beta, v, hw, stage);
         } else {
             update_chunk(p, gi, mat, row, col0, alpha, beta, v, hw, lw, stage);
         }
