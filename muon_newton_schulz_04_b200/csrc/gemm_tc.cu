@@ -236,66 +236,72 @@ __device__ __forceinline__ void update_chunk(const GemmParams& p, const GemmGrou
     stage_chunk(v, stage);
     const EwSeg* sg = p.apply_mode != 0 ? &p.segs[gi.mat_base + mat] : nullptr;
     const bool apply_t = sg != nullptr && sg->transposed;
-    float res[4][8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         const int r = row_w + lr + 8 * i, c = col0 + lc;
-        float acc8[8];
+        float* slot = stage + (lr + 8 * i) * STAGE_LD + lc;     // this lane's 8 words of row lr + 8i
+        float acc8[8], res[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            acc8[k] = stage[(lr + 8 * i) * STAGE_LD + lc + k];
-            res[i][k] = 0.f;
+            acc8[k] = slot[k];
+            res[k] = 0.f;
         }
-        if (r >= gi.m) continue;
-        const size_t o = (size_t)mat * gi.m * gi.ldn + (size_t)r * gi.ldn + c;
-        __nv_bfloat16* hout = gi.xb[p.parity ^ 1] + o;
-        __nv_bfloat16* lout = gi.xlo_out + o;
-        if (c + 7 < gi.n) {
-            const uint32_t h4[4] = {hw[i].x, hw[i].y, hw[i].z, hw[i].w};
-            const uint32_t l4[4] = {lw[i].x, lw[i].y, lw[i].z, lw[i].w};
-            uint32_t ho[4], lo[4];
+        if (r < gi.m) {
+            const size_t o = (size_t)mat * gi.m * gi.ldn + (size_t)r * gi.ldn + c;
+            __nv_bfloat16* hout = gi.xb[p.parity ^ 1] + o;
+            __nv_bfloat16* lout = gi.xlo_out + o;
+            if (c + 7 < gi.n) {
+                const uint32_t h4[4] = {hw[i].x, hw[i].y, hw[i].z, hw[i].w};
+                const uint32_t l4[4] = {lw[i].x, lw[i].y, lw[i].z, lw[i].w};
+                uint32_t ho[4], lo[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float x0 = bf16_bits_lo(h4[e]) + bf16_bits_lo(l4[e]);
-                const float x1 = bf16_bits_hi(h4[e]) + bf16_bits_hi(l4[e]);
-                const float y0 = alpha * acc8[2 * e] + beta * x0;
-                const float y1 = alpha * acc8[2 * e + 1] + beta * x1;
-                const __nv_bfloat162 hh = __floats2bfloat162_rn(y0, y1);
-                const float2 hf = __bfloat1622float2(hh);
-                const __nv_bfloat162 ll = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
-                ho[e] = *reinterpret_cast<const uint32_t*>(&hh);
-                lo[e] = *reinterpret_cast<const uint32_t*>(&ll);
-                // the stored pair is the result: the weight update uses exactly it
-                const float2 lf = __bfloat1622float2(ll);
-                res[i][2 * e] = hf.x + lf.x;
-                res[i][2 * e + 1] = hf.y + lf.y;
-            }
-            *reinterpret_cast<uint4*>(hout) = make_uint4(ho[0], ho[1], ho[2], ho[3]);
-            *reinterpret_cast<uint4*>(lout) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        } else {
-            const __nv_bfloat16* hin = gi.xb[p.parity] + o;
-            const __nv_bfloat16* lin = gi.xlo_in + o;
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = bf16_bits_lo(h4[e]) + bf16_bits_lo(l4[e]);
+                    const float x1 = bf16_bits_hi(h4[e]) + bf16_bits_hi(l4[e]);
+                    const float y0 = alpha * acc8[2 * e] + beta * x0;
+                    const float y1 = alpha * acc8[2 * e + 1] + beta * x1;
+                    const __nv_bfloat162 hh = __floats2bfloat162_rn(y0, y1);
+                    const float2 hf = __bfloat1622float2(hh);
+                    const __nv_bfloat162 ll = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
+                    ho[e] = *reinterpret_cast<const uint32_t*>(&hh);
+                    lo[e] = *reinterpret_cast<const uint32_t*>(&ll);
+                }
+                *reinterpret_cast<uint4*>(hout) = make_uint4(ho[0], ho[1], ho[2], ho[3]);
+                *reinterpret_cast<uint4*>(lout) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                if (sg != nullptr) {
+                    // the stored pair is the result: the weight update uses exactly it
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                if (c + k >= gi.n) continue;
-                const float y = alpha * acc8[k] + beta * (__bfloat162float(hin[k]) + __bfloat162float(lin[k]));
-                const __nv_bfloat16 hh = __float2bfloat16_rn(y);
-                const __nv_bfloat16 ll = __float2bfloat16_rn(y - __bfloat162float(hh));
-                hout[k] = hh;
-                lout[k] = ll;
-                res[i][k] = __bfloat162float(hh) + __bfloat162float(ll);
+                    for (int e = 0; e < 4; ++e) {
+                        res[2 * e] = bf16_bits_lo(ho[e]) + bf16_bits_lo(lo[e]);
+                        res[2 * e + 1] = bf16_bits_hi(ho[e]) + bf16_bits_hi(lo[e]);
+                    }
+                }
+            } else {
+                const __nv_bfloat16* hin = gi.xb[p.parity] + o;
+                const __nv_bfloat16* lin = gi.xlo_in + o;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    if (c + k >= gi.n) continue;
+                    const float y = alpha * acc8[k] + beta * (__bfloat162float(hin[k]) + __bfloat162float(lin[k]));
+                    const __nv_bfloat16 hh = __float2bfloat16_rn(y);
+                    const __nv_bfloat16 ll = __float2bfloat16_rn(y - __bfloat162float(hh));
+                    hout[k] = hh;
+                    lout[k] = ll;
+                    res[k] = __bfloat162float(hh) + __bfloat162float(ll);
+                }
             }
+            if (sg != nullptr && !apply_t) apply_run8(p, *sg, gi.n, r, c, res);
         }
-        if (sg != nullptr && !apply_t) apply_run8(p, *sg, gi.n, r, c, res[i]);
+        // a transposed matrix's W update goes back through this lane's own words of
+        // the buffer (no other lane reads or writes them in between)
+        if (apply_t) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) slot[k] = res[k];
+        }
     }
     if (apply_t) {
-        // W[c][r] of a transposed matrix: back to one row per lane, where the warp's
-        // lanes are 32 consecutive elements of one row of W
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-            for (int k = 0; k < 8; ++k) stage[(lr + 8 * i) * STAGE_LD + lc + k] = res[i][k];
+        // W[c][r]: back to one row per lane, where the warp's lanes are 32
+        // consecutive elements of one row of W
         __syncwarp();
         float val[32];
 #pragma unroll
