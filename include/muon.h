@@ -114,6 +114,17 @@ muon_status muon_create(const muon_config* cfg, int device, muon_handle** out);
 /* Replaces the hyperparameters of a handle (validated first). */
 muon_status muon_set_config(muon_handle* h, const muon_config* cfg);
 
+/* Caps the device memory the handle may hold (workspace, host-step staging and
+ * phase scratch together) at `bytes`; 0 removes the cap.  Buffers already held
+ * are kept.  A later call whose buffers would grow past the cap returns
+ * MUON_ERR_OOM before it launches anything, leaving W, B and the caller's other
+ * buffers untouched; the handle stays usable (raise the cap, or call with fewer
+ * matrices).  MUON_ERR_INVALID for a NULL handle. */
+muon_status muon_set_memory_limit(muon_handle* h, size_t bytes);
+
+/* Device bytes the handle holds now (*bytes).  MUON_ERR_INVALID for NULL arguments. */
+muon_status muon_memory_held(const muon_handle* h, size_t* bytes);
+
 /* One Muon step for every matrix of every group (section 4 eqs. 1-5, eq. 3 with
  * result 2's decay and scale).  Device pointers.  Work is enqueued on `stream`
  * (a cudaStream_t; NULL = legacy default stream). */

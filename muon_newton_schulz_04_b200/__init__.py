@@ -62,6 +62,8 @@ _SIGNATURES = {
     "muon_validate_groups": (ctypes.c_int, [ctypes.POINTER(_Group), ctypes.c_int]),
     "muon_create": (ctypes.c_int, [ctypes.POINTER(MuonConfig), ctypes.c_int, ctypes.POINTER(ctypes.c_void_p)]),
     "muon_set_config": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(MuonConfig)]),
+    "muon_set_memory_limit": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_size_t]),
+    "muon_memory_held": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_size_t)]),
     "muon_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_Group), ctypes.c_int, ctypes.c_void_p]),
     "muon_step_host": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_Group), ctypes.c_int, ctypes.c_void_p]),
     "muon_orthogonalize": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_OrthoGroup), ctypes.c_int, ctypes.c_void_p]),
@@ -203,6 +205,16 @@ class Muon:
     # ------------------------------------------------------------------ API
     def set_config(self, cfg: MuonConfig):
         self._check(lib().muon_set_config(self._h, ctypes.byref(cfg)), "muon_set_config")
+
+    def set_memory_limit(self, nbytes: int):
+        """Caps the device bytes the handle may hold (0: no cap); a call that would grow
+        past it raises MuonError (MUON_ERR_OOM) before launching anything."""
+        self._check(lib().muon_set_memory_limit(self._h, int(nbytes)), "muon_set_memory_limit")
+
+    def memory_held(self) -> int:
+        n = ctypes.c_size_t(0)
+        self._check(lib().muon_memory_held(self._h, ctypes.byref(n)), "muon_memory_held")
+        return n.value
         self.cfg = cfg
 
     def step(self, groups: List[Group], stream=None):

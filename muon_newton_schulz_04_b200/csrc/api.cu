@@ -84,6 +84,7 @@ struct muon_handle {
     DevBuf ws;            // plan workspace
     DevBuf staging;       // muon_step_host staging
     DevBuf scratch;       // muon_ns_phase_run descriptors
+    size_t mem_limit = 0;  // cap on ws + staging + scratch (0: none), muon_set_memory_limit
     int* d_err = nullptr;
     Plan plan;
     EncodeTiledFn encode = nullptr;
@@ -237,6 +238,10 @@ muon_status ensure_buf(muon_handle* h, DevBuf& b, size_t bytes) {
         b.ptr = nullptr;
         b.size = 0;
     }
+    const size_t held = h->ws.size + h->staging.size + h->scratch.size;   // b is already released
+    if (h->mem_limit != 0 && held + bytes > h->mem_limit)
+        return fail(h, MUON_ERR_OOM, "device buffers of %zu bytes would exceed the handle's memory limit of %zu bytes",
+                    held + bytes, h->mem_limit);
     cudaError_t e = cudaMalloc(&b.ptr, bytes);
     if (e != cudaSuccess) {
         cudaGetLastError();
@@ -716,6 +721,18 @@ muon_status muon_set_config(muon_handle* h, const muon_config* cfg) {
     h->cfg = *cfg;
     if (plan_changes) h->plan.valid = false;
     h->plan.uploaded.clear();     // ns_steps / scale may change the segment table
+    return MUON_OK;
+}
+
+muon_status muon_set_memory_limit(muon_handle* h, size_t bytes) {
+    if (!h) return MUON_ERR_INVALID;
+    h->mem_limit = bytes;
+    return MUON_OK;
+}
+
+muon_status muon_memory_held(const muon_handle* h, size_t* bytes) {
+    if (!h || !bytes) return MUON_ERR_INVALID;
+    *bytes = h->ws.size + h->staging.size + h->scratch.size;
     return MUON_OK;
 }
 

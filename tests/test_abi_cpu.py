@@ -108,6 +108,10 @@ def test_create_without_gpu_reports_cuda_error():
     assert not h.value
     assert mb.lib().muon_step(None, None, 0, None) == mb.MUON_ERR_INVALID
     assert mb.lib().muon_destroy(None) == mb.MUON_ERR_INVALID
+    assert mb.lib().muon_set_memory_limit(None, 1 << 20) == mb.MUON_ERR_INVALID
+    held = ctypes.c_size_t(7)
+    assert mb.lib().muon_memory_held(None, ctypes.byref(held)) == mb.MUON_ERR_INVALID
+    assert held.value == 7
 
 
 def test_status_strings():

@@ -1,5 +1,5 @@
-"""Host logic of the matrix-sharded step on CPU: LPT ownership, and a gloo
-world-size-2 run whose ranks end with identical weights equal to a
+"""Host logic of the matrix-sharded step on CPU: LPT ownership, and gloo runs at
+world sizes 2 and 3 whose ranks end with identical weights equal to a
 single-process run."""
 import os
 import socket
@@ -44,13 +44,16 @@ def _free_port():
 
 
 @pytest.mark.timeout(300)
-def test_sharded_step_gloo_world2(tmp_path):
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_step_gloo(tmp_path, world):
+    """World 3 gives shards of unequal element counts (the packed buffer is padded
+    to the largest)."""
     steps = 2
-    tmp.spawn(dist_worker.run, args=(2, _free_port(), steps, str(tmp_path)), nprocs=2, join=True)
+    tmp.spawn(dist_worker.run, args=(world, _free_port(), steps, str(tmp_path)), nprocs=world, join=True)
     ref = dist_worker.reference(steps)
-    outs = [torch.load(tmp_path / f"rank{r}.pt") for r in range(2)]
-    assert sorted(outs[0]["own"] + outs[1]["own"]) == list(range(len(dist_worker.SHAPES)))
-    assert outs[0]["own"] and outs[1]["own"]
+    outs = [torch.load(tmp_path / f"rank{r}.pt") for r in range(world)]
+    assert sorted(i for o in outs for i in o["own"]) == list(range(len(dist_worker.SHAPES)))
+    assert all(o["own"] for o in outs)
     for o in outs:
         for w, wr in zip(o["W"], ref):
             assert torch.equal(w, wr)
