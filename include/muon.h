@@ -49,7 +49,8 @@ typedef enum {
     MUON_OK = 0,
     MUON_ERR_INVALID = 1,        /* bad argument: null pointer, size <= 0, bad enum, ...      */
     MUON_ERR_UNSUPPORTED = 2,    /* device is not sm_100, or a layout the kernels do not take  */
-    MUON_ERR_OOM = 3,            /* workspace allocation failed                                */
+    MUON_ERR_OOM = 3,            /* device buffer allocation failed, or would pass the cap set
+                                    by muon_set_memory_limit                                  */
     MUON_ERR_CUDA = 4,           /* a CUDA runtime call or kernel launch failed                */
     MUON_ERR_DEVICE_TIMEOUT = 5  /* a kernel gave up a bounded wait (reported by muon_sync)    */
 } muon_status;
