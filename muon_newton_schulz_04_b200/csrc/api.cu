@@ -17,6 +17,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/muon.h"
 #include "kernels.cuh"
 #include "plan.h"
@@ -176,8 +178,19 @@ struct PhaseTimer {
     }
 };
 
+// Host-side NVTX range (a no-op unless a profiler is attached): one per entry
+// point and one per enqueued phase, named like the timing kinds.
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+const char* const kPhaseNames[MUON_TIMING_KINDS] = {"momentum_norm", "norm_finalize", "gram", "poly", "update", "apply"};
+
 #define TIMED(h, kind, s, expr)                \
     do {                                       \
+        NvtxRange nr_(kPhaseNames[(kind)]);    \
         PhaseTimer pt_((h), (kind), (s));      \
         CUDA_TRY((h), (expr));                 \
         pt_.done();                            \
@@ -738,6 +751,7 @@ muon_status muon_memory_held(const muon_handle* h, size_t* bytes) {
 
 muon_status muon_step(muon_handle* h, const muon_group* groups, int n_groups, void* stream) {
     if (!h) return MUON_ERR_INVALID;
+    NvtxRange nr("muon_step");
     std::string why;
     if (check_groups(groups, n_groups, &why) != MUON_OK) return fail(h, MUON_ERR_INVALID, "%s", why.c_str());
     DeviceGuard dg(h->device);
@@ -747,6 +761,7 @@ muon_status muon_step(muon_handle* h, const muon_group* groups, int n_groups, vo
 
 muon_status muon_step_host(muon_handle* h, const muon_group* groups, int n_groups, void* stream) {
     if (!h) return MUON_ERR_INVALID;
+    NvtxRange nr("muon_step_host");
     std::string why;
     if (check_groups(groups, n_groups, &why) != MUON_OK) return fail(h, MUON_ERR_INVALID, "%s", why.c_str());
     DeviceGuard dg(h->device);
@@ -824,6 +839,7 @@ muon_status muon_step_host(muon_handle* h, const muon_group* groups, int n_group
 
 muon_status muon_orthogonalize(muon_handle* h, const muon_ortho_group* groups, int n_groups, void* stream) {
     if (!h) return MUON_ERR_INVALID;
+    NvtxRange nr("muon_orthogonalize");
     if (!groups || n_groups <= 0) return fail(h, MUON_ERR_INVALID, "groups must be a non-empty array");
     std::vector<int> shapes;
     std::vector<MatPtrs> mp;
