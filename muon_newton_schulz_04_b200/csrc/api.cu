@@ -376,6 +376,18 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
             }
             P.unit_clusters = h->max_clusters;
         }
+        // nothing is launched with a plan that does not cover its outputs exactly once
+        const std::vector<Tile>* lists[3] = {&tg, &tp, &tu};
+        for (int ph = 0; ph < 3; ++ph) {
+            std::vector<int> kb;
+            for (const Tile& t : *lists[ph]) {
+                const GroupDims& d = P.dims[t.group];
+                kb.push_back(((ph == 0 ? d.n : d.m) + TC_BK - 1) / TC_BK);
+            }
+            const std::string bad = check_plan(P.dims, ph, bm, bn, TC_BK, *lists[ph], kb,
+                                               h->pair ? &upl[ph] : nullptr, h->pair ? h->max_clusters : 1);
+            if (!bad.empty()) return fail(h, MUON_ERR_INVALID, "plan check failed (phase %d): %s", ph, bad.c_str());
+        }
     }
     P.n_gram = (int)tg.size(); P.n_poly = (int)tp.size(); P.n_upd = (int)tu.size();
     const size_t o_tg = take(tg.size() * sizeof(int4) + 16), o_tp = take(tp.size() * sizeof(int4) + 16),
@@ -1126,6 +1138,10 @@ muon_status muon_plan_tiles(const int* shapes, int n_groups, int phase, int* out
     }
     const int pair = tc_gemm_default_pair();
     std::vector<Tile> t = build_tiles(dims, phase, tc_gemm_tile_m(pair), tc_gemm_tile_n(pair));
+    std::vector<int> kb;
+    for (const Tile& x : t) kb.push_back(((phase == 0 ? dims[x.group].n : dims[x.group].m) + TC_BK - 1) / TC_BK);
+    if (!check_plan(dims, phase, tc_gemm_tile_m(pair), tc_gemm_tile_n(pair), TC_BK, t, kb, nullptr, 1).empty())
+        return MUON_ERR_INVALID;
     *n_tiles = (int)t.size();
     if (!out || cap < (int)t.size()) return MUON_ERR_INVALID;
     for (size_t i = 0; i < t.size(); ++i) {
@@ -1147,6 +1163,8 @@ muon_status muon_plan_units(const int* shapes, int n_groups, int phase, int clus
     std::vector<int> kb;
     for (const Tile& x : t) kb.push_back(((phase == 0 ? dims[x.group].n : dims[x.group].m) + TC_BK - 1) / TC_BK);
     UnitPlan up = build_units(t, kb, clusters, split != 0, split == 0);
+    if (!check_plan(dims, phase, tc_gemm_tile_m(1), tc_gemm_tile_n(1), TC_BK, t, kb, &up, clusters).empty())
+        return MUON_ERR_INVALID;
     *n_units = (int)up.units.size();
     if (!out || cap < (int)up.units.size()) return MUON_ERR_INVALID;
     for (int c = 0; c < clusters; ++c) {

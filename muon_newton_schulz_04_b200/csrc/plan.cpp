@@ -4,6 +4,8 @@
 #include <algorithm>
 #include <cstdlib>
 #include <cstring>
+#include <map>
+#include <tuple>
 
 namespace muon {
 
@@ -119,6 +121,86 @@ UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kbl
         up.begin.push_back((int)up.units.size());
     }
     return up;
+}
+
+std::string check_plan(const std::vector<GroupDims>& groups, int phase, int bm, int bn, int bk,
+                       const std::vector<Tile>& tiles, const std::vector<int>& kblocks, const UnitPlan* up,
+                       int clusters) {
+    using Key = std::tuple<int, int, int, int>;
+    auto msg = [](const char* what, long long i) { return std::string(what) + " (entry " + std::to_string(i) + ")"; };
+    if (kblocks.size() != tiles.size()) return "one K-block count per tile expected";
+    long long expected = 0;
+    for (const GroupDims& d : groups) {
+        const int out_cols = (phase == 2) ? d.n : d.m;
+        const long long tr = (d.m + bm - 1) / bm, tc = (out_cols + bn - 1) / bn;
+        long long per = 0;
+        for (long long i = 0; i < tr; ++i)
+            for (long long j = 0; j < tc; ++j)
+                if (phase == 2 || std::min((j + 1) * bn, (long long)d.m) - 1 >= i * bm) ++per;
+        expected += per * d.count;
+    }
+    if ((long long)tiles.size() != expected) return "tile count differs from the shapes' tile count";
+    std::map<Key, int> index;
+    for (size_t i = 0; i < tiles.size(); ++i) {
+        const Tile& t = tiles[i];
+        if (t.group < 0 || t.group >= (int)groups.size()) return msg("tile group out of range", i);
+        const GroupDims& d = groups[t.group];
+        const int out_cols = (phase == 2) ? d.n : d.m;
+        if (t.mat < 0 || t.mat >= d.count) return msg("tile matrix out of range", i);
+        if (t.tile_row < 0 || (long long)t.tile_row * bm >= d.m) return msg("tile row out of range", i);
+        if (t.tile_col < 0 || (long long)t.tile_col * bn >= out_cols) return msg("tile column out of range", i);
+        if (phase != 2 && std::min((long long)(t.tile_col + 1) * bn, (long long)d.m) - 1 < (long long)t.tile_row * bm)
+            return msg("symmetric tile entirely below the diagonal", i);
+        const int k = (phase == 0) ? d.n : d.m;
+        if (kblocks[i] != (k + bk - 1) / bk) return msg("wrong K-block count", i);
+        if (!index.emplace(Key{t.group, t.mat, t.tile_row, t.tile_col}, (int)i).second) return msg("duplicate tile", i);
+    }
+    if (up == nullptr) return "";
+    const std::vector<Unit>& us = up->units;
+    if ((int)up->begin.size() != clusters + 1 || up->begin.front() != 0 || up->begin.back() != (int)us.size())
+        return "cluster offsets do not span the unit list";
+    for (int c = 0; c < clusters; ++c)
+        if (up->begin[c] > up->begin[c + 1]) return msg("cluster offsets decrease", c);
+    std::vector<std::vector<int>> of(tiles.size());
+    for (size_t i = 0; i < us.size(); ++i) {
+        const Unit& u = us[i];
+        auto it = index.find(Key{u.tile.group, u.tile.mat, u.tile.tile_row, u.tile.tile_col});
+        if (it == index.end()) return msg("unit of a tile not in the list", i);
+        const int kb = kblocks[it->second];
+        if (u.k_begin < 0 || u.k_begin >= u.k_end || u.k_end > kb) return msg("unit K range outside its tile", i);
+        if (u.kind < 0 || u.kind > 2 || u.n_half < 0 || u.n_half > 2) return msg("unit kind or half out of range", i);
+        if (u.n_half != 0 && (u.kind != 0 || u.k_begin != 0 || u.k_end != kb)) return msg("column half is not a whole-K unit", i);
+        if (u.kind == 1 && (u.k_begin != 0 || u.nslots < 1)) return msg("split head does not start at K-block 0", i);
+        if (u.kind != 0 && (u.slot < 0 || u.slot + (u.kind == 1 ? u.nslots : 1) > up->nslots))
+            return msg("partial-sum slot out of range", i);
+        of[it->second].push_back((int)i);
+    }
+    for (size_t t = 0; t < tiles.size(); ++t) {
+        std::vector<int> l = of[t];
+        const int kb = kblocks[t];
+        if (l.empty()) return msg("tile without a unit", t);
+        if (l.size() == 1) {
+            const Unit& u = us[l[0]];
+            if (u.kind != 0 || u.n_half != 0 || u.k_begin != 0 || u.k_end != kb) return msg("single unit is not the whole tile", t);
+            continue;
+        }
+        if (us[l[0]].n_half != 0) {
+            if (l.size() != 2 || us[l[0]].n_half + us[l[1]].n_half != 3 || us[l[1]].n_half == 0)
+                return msg("column halves do not pair up", t);
+            continue;
+        }
+        std::sort(l.begin(), l.end(), [&](int a, int b) { return us[a].k_begin < us[b].k_begin; });
+        const Unit& head = us[l[0]];
+        if (head.kind != 1 || head.nslots != (int)l.size() - 1) return msg("split tile without a matching head", t);
+        for (size_t i = 1; i < l.size(); ++i) {
+            const Unit& u = us[l[i]];
+            if (u.kind != 2 || u.n_half != 0) return msg("split part of the wrong kind", t);
+            if (u.k_begin != us[l[i - 1]].k_end) return msg("split parts leave a gap or overlap", t);
+            if (u.slot != head.slot + (int)i - 1) return msg("split part slot out of order", t);
+        }
+        if (us[l.back()].k_end != kb) return msg("split parts stop before the last K-block", t);
+    }
+    return "";
 }
 
 int tc_gemm_split_tiles() {

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cstdint>
+#include <string>
 #include <vector>
 
 namespace muon {
@@ -54,6 +55,17 @@ struct UnitPlan {
 // one per cluster, so the last round takes about half as long.
 UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kblocks, int clusters, bool split,
                      bool half_tail = false);
+
+// Host-side check of a plan before anything is launched with it: the tile list of
+// `phase` holds every tile it should exactly once (in range, and for GRAM / POLY
+// touching col >= row), kblocks[i] is tile i's K-block count, and -- when `up` is
+// given -- the units of `clusters` clusters cover each tile exactly once: one whole
+// unit, two column halves, or a head (kind 1, from K-block 0) and kind-2 parts that
+// continue its K range without gaps, with consistent partial-sum slots.  Returns an
+// empty string when the plan is valid, else what is wrong.
+std::string check_plan(const std::vector<GroupDims>& groups, int phase, int bm, int bn, int bk,
+                       const std::vector<Tile>& tiles, const std::vector<int>& kblocks, const UnitPlan* up,
+                       int clusters);
 
 // 0 unless the environment variable MUON_GEMM_SPLIT is "1": split the K-blocks of
 // the last, partial round of tiles over all clusters (build_units).  Off by
