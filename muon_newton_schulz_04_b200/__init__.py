@@ -205,6 +205,7 @@ class Muon:
     # ------------------------------------------------------------------ API
     def set_config(self, cfg: MuonConfig):
         self._check(lib().muon_set_config(self._h, ctypes.byref(cfg)), "muon_set_config")
+        self.cfg = cfg
 
     def set_memory_limit(self, nbytes: int):
         """Caps the device bytes the handle may hold (0: no cap); a call that would grow
@@ -215,7 +216,6 @@ class Muon:
         n = ctypes.c_size_t(0)
         self._check(lib().muon_memory_held(self._h, ctypes.byref(n)), "muon_memory_held")
         return n.value
-        self.cfg = cfg
 
     def step(self, groups: List[Group], stream=None):
         arr, keep = self._groups(groups, True)
