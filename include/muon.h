@@ -84,7 +84,9 @@ typedef struct {
 /* Same-shape matrices.  W: fp32 rows x cols (updated in place); G: gradient,
  * bf16 or fp32 (read only); B: fp32 momentum (updated in place; zero before the
  * first step).  All device pointers, 4-byte aligned at least; 16-byte aligned
- * pointers and cols % 8 == 0 take the vectorised path. */
+ * pointers and cols % 8 == 0 take the vectorised path.  W and B are written, so no
+ * W or B may share memory with any W, G or B of the call (MUON_ERR_INVALID); one
+ * gradient buffer may be given for several matrices. */
 typedef struct {
     int rows, cols, count;
     int grad_dtype;          /* muon_dtype */

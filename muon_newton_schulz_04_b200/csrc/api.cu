@@ -8,6 +8,7 @@
 //
 // All launches go to the caller's stream; nothing here synchronises except the
 // entry points documented to do so.
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstdarg>
@@ -239,6 +240,32 @@ muon_status check_groups(const muon_group* g, int n, std::string* why) {
         total += g[i].count;
     }
     if (total > (1 << 24)) { *why = "too many matrices"; return MUON_ERR_INVALID; }
+    // W and B are written in place: neither may overlap any other matrix's W, G or B
+    // (G buffers are only read and may be shared).
+    struct Span { uintptr_t a, b; bool written; int group, index; char what; };
+    std::vector<Span> sp;
+    sp.reserve((size_t)total * 3);
+    for (int i = 0; i < n; ++i) {
+        const uintptr_t e = (uintptr_t)g[i].rows * (uintptr_t)g[i].cols;
+        const uintptr_t gb = e * (g[i].grad_dtype == MUON_BF16 ? 2 : 4);
+        for (int k = 0; k < g[i].count; ++k) {
+            const uintptr_t w = (uintptr_t)g[i].W[k], b = (uintptr_t)g[i].B[k], gg = (uintptr_t)g[i].G[k];
+            sp.push_back(Span{w, w + 4 * e, true, i, k, 'W'});
+            sp.push_back(Span{b, b + 4 * e, true, i, k, 'B'});
+            sp.push_back(Span{gg, gg + gb, false, i, k, 'G'});
+        }
+    }
+    std::sort(sp.begin(), sp.end(), [](const Span& x, const Span& y) { return x.a < y.a; });
+    uintptr_t end_any = 0, end_written = 0;
+    for (const Span& x : sp) {
+        if (x.a < end_written || (x.written && x.a < end_any)) {
+            *why = "group " + std::to_string(x.group) + ": " + x.what + "[" + std::to_string(x.index) +
+                   "] overlaps a buffer that the step writes (W and B must not share memory with any W, G or B)";
+            return MUON_ERR_INVALID;
+        }
+        end_any = std::max(end_any, x.b);
+        if (x.written) end_written = std::max(end_written, x.b);
+    }
     return MUON_OK;
 }
 

@@ -241,3 +241,31 @@ def test_default_units_cover_each_tile_once(shapes, clusters, phase):
 def test_no_undefined_library_symbols():
     out = os.popen(f"nm -D --undefined-only {mb.LIB_PATH}").read()
     assert "muon" not in out
+
+
+def test_group_validation_rejects_overlapping_written_buffers():
+    """W and B are updated in place: they may not share memory with any W, G or B of
+    the call.  Gradients are only read and may be shared."""
+    L = mb.lib()
+    ok_cases = [dict(w=[0x10000, 0x10080]),                     # 4 x 8 fp32 = 128 B: adjacent is fine
+                dict(g=[0x300000, 0x300000]),                   # one gradient read by both matrices
+                dict(g=[0x300000, 0x300020])]                   # bf16 gradients overlapping each other
+    for kw in ok_cases:
+        g, keep = _group(**kw)
+        assert L.muon_validate_groups(ctypes.byref(g), 1) == mb.MUON_OK, kw
+    bad_cases = [dict(w=[0x10000, 0x10000]),                    # the same W twice
+                 dict(w=[0x10000, 0x10040]),                    # partial overlap of two W
+                 dict(b=[0x10000, 0x211000]),                   # B[0] is W[0]
+                 dict(g=[0x10000, 0x300000]),                   # G[0] is W[0]
+                 dict(g=[0x210040, 0x300000])]                  # G[0] inside B[0] (at 0x210000)
+    for kw in bad_cases:
+        g, keep = _group(**kw)
+        assert L.muon_validate_groups(ctypes.byref(g), 1) == mb.MUON_ERR_INVALID, kw
+    # across groups: the second group's W is the first group's B[1] (at 0x211000)
+    g1, k1 = _group()
+    g2, k2 = _group(count=1, w=[0x211000], g=[0x500000], b=[0x600000])
+    arr = (mb._Group * 2)(g1, g2)
+    assert L.muon_validate_groups(arr, 2) == mb.MUON_ERR_INVALID
+    g2b, k2b = _group(count=1, w=[0x700000], g=[0x500000], b=[0x600000])
+    arr = (mb._Group * 2)(g1, g2b)
+    assert L.muon_validate_groups(arr, 2) == mb.MUON_OK
