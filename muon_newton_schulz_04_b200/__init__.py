@@ -250,7 +250,15 @@ class Muon:
 
     def qk_clip(self, Wq, Wk, max_logits, head_dim: int, tau: float, stream=None):
         """MuonClip's QK-Clip: rows of head h of Wq and Wk times sqrt(min(1, tau / max_logits[h]))."""
+        import torch
+        for name, t in (("Wq", Wq), ("Wk", Wk), ("max_logits", max_logits)):
+            if t is None and name == "Wk":
+                continue
+            if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
         n_heads = max_logits.numel()
+        if Wq.dim() != 2:
+            raise ValueError("Wq must be 2-D")
         rows, cols = Wq.shape
         if rows != n_heads * head_dim or (Wk is not None and tuple(Wk.shape) != (rows, cols)):
             raise ValueError("Wq / Wk must be (n_heads * head_dim) x cols")

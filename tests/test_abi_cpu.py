@@ -269,3 +269,20 @@ def test_group_validation_rejects_overlapping_written_buffers():
     g2b, k2b = _group(count=1, w=[0x700000], g=[0x500000], b=[0x600000])
     arr = (mb._Group * 2)(g1, g2b)
     assert L.muon_validate_groups(arr, 2) == mb.MUON_OK
+
+
+def test_qk_clip_binding_checks_tensors_before_the_library():
+    """The binding refuses tensors the fp32 kernel cannot read safely (wrong dtype,
+    device or layout, or a head count that does not match the rows) before any call
+    into the library."""
+    import torch
+    opt = mb.Muon.__new__(mb.Muon)               # no device handle: nothing may reach the library
+    opt._h = ctypes.c_void_p()
+    Wq = torch.zeros(8, 4)
+    S = torch.ones(2)
+    with pytest.raises(ValueError):
+        opt.qk_clip(Wq, None, S, 4, 10.0)                          # CPU tensors
+    with pytest.raises(ValueError):
+        opt.qk_clip(Wq.to(torch.bfloat16), None, S, 4, 10.0)       # not float32
+    with pytest.raises(ValueError):
+        opt.qk_clip(torch.zeros(4, 8).t(), None, S, 4, 10.0)       # not contiguous
