@@ -152,12 +152,16 @@ def _dtype_code(t) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def _check_tensors(ts, shape, on_cuda: bool):
+def _check_tensors(ts, shape, on_cuda: bool, dtype=None):
+    """Same shape, dense, on the expected device kind and, when given, of one dtype
+    (the library reads and writes these buffers as dense arrays of that type)."""
     for t in ts:
         if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
             raise ValueError(f"expected contiguous tensors of shape {tuple(shape)}, got {tuple(t.shape)}")
         if t.is_cuda != on_cuda:
             raise ValueError("tensor on the wrong device kind")
+        if dtype is not None and t.dtype != dtype:
+            raise ValueError(f"expected {dtype} tensors, got {t.dtype}")
 
 
 def _stream(stream) -> int:
@@ -188,10 +192,11 @@ class Muon:
         arr = (_Group * len(groups))()
         keep = []
         for i, g in enumerate(groups):
+            import torch
             rows, cols = g.W[0].shape
-            _check_tensors(g.W, (rows, cols), on_cuda)
-            _check_tensors(g.G, (rows, cols), on_cuda)
-            _check_tensors(g.B, (rows, cols), on_cuda)
+            _check_tensors(g.W, (rows, cols), on_cuda, torch.float32)
+            _check_tensors(g.G, (rows, cols), on_cuda, g.G[0].dtype)
+            _check_tensors(g.B, (rows, cols), on_cuda, torch.float32)
             if not (len(g.W) == len(g.G) == len(g.B)):
                 raise ValueError("W, G and B lists differ in length")
             pw, pg, pb = _ptrs(g.W), _ptrs(g.G), _ptrs(g.B)
@@ -219,10 +224,12 @@ class Muon:
 
     def step(self, groups: List[Group], stream=None):
         arr, keep = self._groups(groups, True)
+        self._shapes = [(arr[i].rows, arr[i].cols, arr[i].count) for i in range(len(groups))]
         self._check(lib().muon_step(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream))), "muon_step")
 
     def step_host(self, groups: List[Group], stream=None):
         arr, keep = self._groups(groups, False)
+        self._shapes = [(arr[i].rows, arr[i].cols, arr[i].count) for i in range(len(groups))]
         self._check(lib().muon_step_host(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream))), "muon_step_host")
 
     def orthogonalize(self, groups, stream=None):
@@ -230,9 +237,10 @@ class Muon:
         arr = (_OrthoGroup * len(groups))()
         keep = []
         for i, (Ms, Os) in enumerate(groups):
+            import torch
             rows, cols = Ms[0].shape
-            _check_tensors(Ms, (rows, cols), True)
-            _check_tensors(Os, (rows, cols), True)
+            _check_tensors(Ms, (rows, cols), True, Ms[0].dtype)
+            _check_tensors(Os, (rows, cols), True, torch.float32)
             pm, po = _ptrs(Ms), _ptrs(Os)
             keep += [pm, po]
             arr[i] = _OrthoGroup(rows, cols, len(Ms), _dtype_code(Ms[0]),
@@ -279,6 +287,13 @@ class Muon:
         return list(buf[: n.value])
 
     def last_update(self, group: int, index: int, dst, stream=None):
+        """O of matrix `index` of group `group` of the last step, written to dst (fp32,
+        the matrix's rows x cols, contiguous, on the device)."""
+        import torch
+        shapes = getattr(self, "_shapes", None)
+        if shapes is None or not (0 <= group < len(shapes)) or not (0 <= index < shapes[group][2]):
+            raise ValueError(f"no matrix {index} in group {group} of the last call")
+        _check_tensors([dst], shapes[group][:2], True, torch.float32)
         self._check(lib().muon_last_update(self._h, group, index, ctypes.c_void_p(dst.data_ptr()),
                                            ctypes.c_void_p(_stream(stream))), "muon_last_update")
 

@@ -286,3 +286,22 @@ def test_qk_clip_binding_checks_tensors_before_the_library():
         opt.qk_clip(Wq.to(torch.bfloat16), None, S, 4, 10.0)       # not float32
     with pytest.raises(ValueError):
         opt.qk_clip(torch.zeros(4, 8).t(), None, S, 4, 10.0)       # not contiguous
+
+
+def test_binding_checks_buffer_dtypes_before_the_library():
+    """W and B are read and written as fp32 and the gradients of a group share one
+    dtype; last_update needs an fp32 buffer of the matrix's shape.  The binding
+    refuses anything else before any call into the library."""
+    import torch
+    opt = mb.Muon.__new__(mb.Muon)
+    opt._h = ctypes.c_void_p()
+    W, B = torch.zeros(4, 8), torch.zeros(4, 8)
+    G = torch.zeros(4, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        opt.step_host([mb.Group(W=[W.to(torch.bfloat16)], G=[G], B=[B])])
+    with pytest.raises(ValueError):
+        opt.step_host([mb.Group(W=[W], G=[G], B=[B.double()])])
+    with pytest.raises(ValueError):
+        opt.step_host([mb.Group(W=[W, W.clone()], G=[G, G.float()], B=[B, B.clone()])])
+    with pytest.raises(ValueError):
+        opt.last_update(0, 0, torch.zeros(4, 8))              # no call has recorded any matrix
