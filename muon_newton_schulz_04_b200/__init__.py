@@ -325,10 +325,14 @@ class Muon:
 def momentum_norm_noalloc(G, B, norm_out, U_out=None, momentum: float = 0.95, nesterov: bool = True, stream=None):
     """Momentum phase of one matrix with no device allocation (see muon.h):
     B <- momentum*B + G in place, U_out = G + momentum*B (or B), norm_out[0] = ||U||_F."""
+    import torch
     rows, cols = B.shape
-    _check_tensors([G, B], (rows, cols), True)
+    _check_tensors([G], (rows, cols), True)
+    _check_tensors([B], (rows, cols), True, torch.float32)
     if U_out is not None:
-        _check_tensors([U_out], (rows, cols), True)
+        _check_tensors([U_out], (rows, cols), True, torch.float32)
+    if norm_out.dtype != torch.float32 or not norm_out.is_cuda or norm_out.numel() < 1:
+        raise ValueError("norm_out must be a float32 CUDA tensor with at least one element")
     err = ctypes.create_string_buffer(256)
     st = lib().muon_momentum_norm_noalloc(rows, cols, _dtype_code(G), G.data_ptr(), B.data_ptr(),
                                           None if U_out is None else U_out.data_ptr(), float(momentum), int(nesterov),
