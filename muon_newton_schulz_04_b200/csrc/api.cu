@@ -222,6 +222,28 @@ muon_status check_shape(int rows, int cols, int count, std::string* why) {
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// A buffer of a call: [a, b) bytes, written or only read, and where it came from.
+struct Span { uintptr_t a, b; bool written; int group, index; char what; };
+
+// MUON_ERR_INVALID when a written span overlaps any other span (read-only spans may
+// overlap each other).  One sort and one sweep: a span overlaps an earlier one
+// exactly when it starts before the largest end seen so far.
+muon_status check_spans(std::vector<Span>& sp, std::string* why) {
+    std::sort(sp.begin(), sp.end(), [](const Span& x, const Span& y) { return x.a < y.a; });
+    uintptr_t end_any = 0, end_written = 0;
+    for (const Span& x : sp) {
+        if (x.a < end_written || (x.written && x.a < end_any)) {
+            *why = "group " + std::to_string(x.group) + ": " + x.what + "[" + std::to_string(x.index) +
+                   "] overlaps a buffer that the call writes (written buffers may not share memory with any "
+                   "other buffer of the call)";
+            return MUON_ERR_INVALID;
+        }
+        end_any = std::max(end_any, x.b);
+        if (x.written) end_written = std::max(end_written, x.b);
+    }
+    return MUON_OK;
+}
+
 muon_status check_groups(const muon_group* g, int n, std::string* why) {
     if (!g || n <= 0) { *why = "groups must be a non-empty array"; return MUON_ERR_INVALID; }
     long long total = 0;
@@ -242,7 +264,6 @@ muon_status check_groups(const muon_group* g, int n, std::string* why) {
     if (total > (1 << 24)) { *why = "too many matrices"; return MUON_ERR_INVALID; }
     // W and B are written in place: neither may overlap any other matrix's W, G or B
     // (G buffers are only read and may be shared).
-    struct Span { uintptr_t a, b; bool written; int group, index; char what; };
     std::vector<Span> sp;
     sp.reserve((size_t)total * 3);
     for (int i = 0; i < n; ++i) {
@@ -255,18 +276,7 @@ muon_status check_groups(const muon_group* g, int n, std::string* why) {
             sp.push_back(Span{gg, gg + gb, false, i, k, 'G'});
         }
     }
-    std::sort(sp.begin(), sp.end(), [](const Span& x, const Span& y) { return x.a < y.a; });
-    uintptr_t end_any = 0, end_written = 0;
-    for (const Span& x : sp) {
-        if (x.a < end_written || (x.written && x.a < end_any)) {
-            *why = "group " + std::to_string(x.group) + ": " + x.what + "[" + std::to_string(x.index) +
-                   "] overlaps a buffer that the step writes (W and B must not share memory with any W, G or B)";
-            return MUON_ERR_INVALID;
-        }
-        end_any = std::max(end_any, x.b);
-        if (x.written) end_written = std::max(end_written, x.b);
-    }
-    return MUON_OK;
+    return check_spans(sp, why);
 }
 
 muon_status ensure_buf(muon_handle* h, DevBuf& b, size_t bytes) {
@@ -895,6 +905,21 @@ muon_status muon_orthogonalize(muon_handle* h, const muon_ortho_group* groups, i
                 return fail(h, MUON_ERR_INVALID, "group %d: misaligned pointer at %d", i, k);
             mp.push_back(MatPtrs{groups[i].M[k], nullptr, groups[i].O[k], groups[i].in_dtype == MUON_BF16 ? 1 : 0, 1.0f});
         }
+    }
+    {
+        // O is written: it may not overlap any M or O of the call
+        std::vector<Span> sp;
+        for (int i = 0; i < n_groups; ++i) {
+            const uintptr_t e = (uintptr_t)groups[i].rows * (uintptr_t)groups[i].cols;
+            const uintptr_t mb = e * (groups[i].in_dtype == MUON_BF16 ? 2 : 4);
+            for (int k = 0; k < groups[i].count; ++k) {
+                const uintptr_t m = (uintptr_t)groups[i].M[k], o = (uintptr_t)groups[i].O[k];
+                sp.push_back(Span{m, m + mb, false, i, k, 'M'});
+                sp.push_back(Span{o, o + 4 * e, true, i, k, 'O'});
+            }
+        }
+        std::string why;
+        if (check_spans(sp, &why) != MUON_OK) return fail(h, MUON_ERR_INVALID, "%s", why.c_str());
     }
     DeviceGuard dg(h->device);
     h->last_error.clear();
