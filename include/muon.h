@@ -142,7 +142,8 @@ muon_status muon_step_host(muon_handle* h, const muon_group* groups, int n_group
 /* Orthogonalisation alone: O = NS_k(M / (||M||_F + eps)) per matrix, with the
  * orientation rule of section 4 and the handle's ns_steps / coefficients /
  * precision.  M: bf16 or fp32 rows x cols (device, read only); O: fp32 rows x cols
- * (device, written).  Same conventions as muon_group. */
+ * (device, written; it may not overlap any M or O of the call).  Same conventions
+ * as muon_group. */
 typedef struct {
     int rows, cols, count;
     int in_dtype;            /* muon_dtype */
