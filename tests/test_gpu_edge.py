@@ -161,6 +161,10 @@ def test_step_argument_errors():
         opt.step([mb.Group(W=[W], G=[torch.zeros(8, 8, dtype=torch.float16, device="cuda")], B=[W])])
     with pytest.raises(ValueError):
         opt.step([mb.Group(W=[W], G=[torch.zeros(8, 9, device="cuda")], B=[W])])
+    G8 = torch.zeros(8, 8, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(mb.MuonError) as e:                  # B is W: refused before any launch
+        opt.step([mb.Group(W=[W], G=[G8], B=[W])])
+    assert e.value.status == mb.MUON_ERR_INVALID
     bad = mb.config()
     bad.momentum = 2.0
     with pytest.raises(mb.MuonError) as e:
