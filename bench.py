@@ -145,11 +145,14 @@ class ClockSampler:
 def elementwise_bytes(w: wl.Workload):
     """Algorithmic HBM bytes of the two memory-bound kernels of one step.
 
-    momentum+norm: read G (2 or 4 B) and B (4 B), write B (4 B) and the iterate as
-    a bf16 pair hi + lo (2 + 2 B) = 14 B/elem for bf16 gradients.
-    apply (when not fused): read W (4 B) and O = hi + lo (4 B), write W (4 B) = 12 B/elem."""
+    momentum+norm, the method's count: read G (2 B bf16, 4 B fp32) and B (4 B), write
+    B (4 B) and the bf16 iterate X0 (2 B) = 12 B/elem for bf16 gradients (14 B for
+    fp32 ones).  This library also writes the low half of its bf16-pair iterate
+    (X0 = hi + lo, 2 B more), reported separately as the bytes it moves.
+    apply (when not fused): read W (4 B) and O = hi + lo (4 B), write W (4 B) = 12 B/elem.
+    Returns (momentum algorithmic, momentum moved, apply)."""
     g = 2 if w.grad_dtype == wl.BF16 else 4
-    return w.elements * (g + 4 + 4 + 2 + 2), w.elements * 12
+    return w.elements * (g + 4 + 4 + 2), w.elements * (g + 4 + 4 + 2 + 2), w.elements * 12
 
 
 def update_gemm_flops(w: wl.Workload):
@@ -282,6 +285,133 @@ def run_reference(args, w):
     return 0
 
 
+def measure(opt, groups, steps: int, warmup: int, world: int, dev, load_s: float, clock_gpu: int):
+    """Warm-up, a burst run, then `steps` timed steps inside a load window of
+    `load_s` seconds that the clock sampler sees, then the same steps again with the
+    library's per-launch events.  Returns (ms per step, burst ms per step, phases,
+    clocks)."""
+    import torch
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        opt.step(groups)
+    opt.sync()
+    # burst: the same K steps right after warm-up, before the power cap engages
+    # (too short for the 200 ms clock sampler; reported beside the main number)
+    eb0, eb1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    eb0.record(stream)
+    for _ in range(steps):
+        opt.step(groups)
+    eb1.record(stream)
+    torch.cuda.synchronize()
+    burst_ms = max_over_ranks(eb0.elapsed_time(eb1), world, dev) / steps
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(clock_gpu)
+    clocks.start()
+    t_load = time.perf_counter()
+    while time.perf_counter() - t_load < load_s:
+        for _ in range(4):
+            opt.step(groups)
+        torch.cuda.synchronize()
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    ev0.record(stream)
+    for _ in range(steps):
+        opt.step(groups)
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    ms_total = ev0.elapsed_time(ev1)
+    # per-kernel times: the same K steps again with the library's per-launch events
+    # (kept out of the main timed region: events between launches stop the next
+    # kernel's prologue from overlapping the previous kernel's tail)
+    opt.timing(True)
+    opt.timing_read()
+    for _ in range(steps):
+        opt.step(groups)
+    phases = opt.timing_read()
+    opt.timing(False)
+    t_load = time.perf_counter()
+    while time.perf_counter() - t_load < 0.4 * load_s:
+        for _ in range(4):
+            opt.step(groups)
+        torch.cuda.synchronize()
+    clk = clocks.stop()
+    ms_total = max_over_ranks(ms_total, world, dev)
+    return ms_total / steps, burst_ms, phases, clk
+
+
+def ns_figures(w: wl.Workload, ms_step: float, burst_ms: float, phases, steps: int, peaks, world: int = 1):
+    """Newton-Schulz throughput on both FLOP counts and the momentum kernel's HBM
+    throughput, each with the numbers it is computed from.
+
+    nominal:   5 (4 m^2 n + 2 m^3) per matrix (the metric's count), over the step time;
+    symmetric: 5 (3 m^2 n + m^3), the work left when the two symmetric products are
+               formed on one triangle, over the step time minus the momentum kernel's
+               time (the Newton-Schulz part of the step); its fraction of the bf16
+               dense peak is the roofline fraction of the Newton-Schulz GEMMs;
+    phase sum: nominal FLOPs over the sum of the event-bracketed GEMM launches (events
+               between launches defeat the overlap of one kernel's prologue with the
+               previous one's tail, so the sum is longer than the step's share)."""
+    flops_nom, flops_sym = w.ns_flops_nominal(), w.ns_flops_symmetric()
+    mom_ms = phases["momentum_norm"][0] / max(phases["momentum_norm"][1], 1)
+    gemm_ms = sum(phases[k][0] for k in ("gram", "poly", "update")) / steps
+    ns_ms = max(ms_step - mom_ms, 1e-9)
+    ns_burst_ms = max(burst_ms - mom_ms, 1e-9)
+    b_mom, b_mom_moved, _ = elementwise_bytes(w)
+    sym = flops_sym / (ns_ms * 1e-3) / 1e12
+    return {
+        "ns5_tflops_nominal": round(flops_nom * world / (ms_step * 1e-3) / 1e12, 2),
+        "ns5_symmetric": {
+            "tflops": round(sym, 2),
+            "frac_sustained": round(sym / peaks["bf16_tflops_sustained"], 4),
+            "tflops_burst": round(flops_sym / (ns_burst_ms * 1e-3) / 1e12, 2),
+            "frac_burst": round(flops_sym / (ns_burst_ms * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+            "flops_per_step": flops_sym, "ns_ms_per_step": round(ns_ms, 4),
+            "basis": "5(3m^2n+m^3) FLOPs / (ms_per_step - momentum kernel ms); burst: same with the burst step time"},
+        "ns5_tflops_phase_sum": round(flops_nom / (gemm_ms * 1e-3) / 1e12, 2),
+        "momentum_ms": round(mom_ms, 4),
+        "momentum_gbs": round(b_mom / (mom_ms * 1e-3) / 1e9, 1),
+        "momentum_frac_of_hbm": round(b_mom / (mom_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "momentum_bytes_per_elem": b_mom / w.elements,
+        "momentum_gbs_moved": round(b_mom_moved / (mom_ms * 1e-3) / 1e9, 1),
+        "momentum_moved_bytes_per_elem": b_mom_moved / w.elements,
+    }
+
+
+def per_workload_rows(args, world, dev, peaks, local, skip_key):
+    """One row per other workload, drawn on the device (workloads.device_tensors)."""
+    import torch
+    import muon_newton_schulz_04_b200 as mb
+    rows = []
+    for key in ("tiny", "gpt2_small", "square4096", "gpt2_xl", "moe_sweep"):
+        if key == skip_key:
+            continue
+        w = wl.get(key)
+        cfg = mb.config(lr=w.lr, momentum=w.momentum, nesterov=int(w.nesterov), weight_decay=w.weight_decay,
+                        ns_steps=w.ns_steps, eps=w.eps, precision=mb.PREC_BF16)
+        opt = mb.Muon(cfg, device=local)
+        W, G = wl.device_tensors(w, 0, dev)
+        B = [torch.zeros_like(x) for x in W]
+        groups = groups_of(w, W, G, B)
+        steps = max(5, min(args.steps, 10))
+        ms, burst, phases, clk = measure(opt, groups, steps, 3, world, dev, 0.5, local)
+        row = {"workload": key, "matrices": w.count, "elements": w.elements, "steps": steps,
+               "ms_per_step": round(ms, 4), "burst_ms_per_step": round(burst, 4)}
+        row.update(ns_figures(w, ms, burst, phases, steps, peaks, world))
+        row["phase_ms_per_step"] = {k: round(v[0] / steps, 4) for k, v in phases.items()}
+        row["gpu_launches_per_step"] = sum(n for (_, n) in phases.values()) // steps
+        row["clocks"] = clk
+        row["inputs"] = "drawn on the device (workloads.device_tensors: same recipe, torch generator)"
+        rows.append(row)
+        opt.close()
+        del W, G, B, groups
+        torch.cuda.empty_cache()
+    return rows
+
+
 def run_ours(args, w):
     import torch
     import muon_newton_schulz_04_b200 as mb
@@ -301,66 +431,13 @@ def run_ours(args, w):
     groups = groups_of(w, W, G, B)
     stream = torch.cuda.current_stream()
 
-    for _ in range(args.warmup):
-        opt.step(groups)
-    opt.sync()
-
-    # --- burst: the same K steps right after warm-up, before the power cap engages
-    # (too short for the 200 ms clock sampler; reported beside the main number)
-    eb0, eb1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world, dev)
-    torch.cuda.synchronize()
-    eb0.record(stream)
-    for _ in range(args.steps):
-        opt.step(groups)
-    eb1.record(stream)
-    torch.cuda.synchronize()
-    burst_ms = max_over_ranks(eb0.elapsed_time(eb1), world, dev) / args.steps
-
-    # --- device-resident timed region, inside an untimed load window so that the
-    # clock sampler (200 ms period) sees the GPU under this load during it
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
-    clocks.start()
-    t_load = time.perf_counter()
-    while time.perf_counter() - t_load < 1.0:
-        for _ in range(10):
-            opt.step(groups)
-        torch.cuda.synchronize()
-    barrier(world, dev)
-    torch.cuda.synchronize()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        opt.step(groups)
-    ev1.record(stream)
-    torch.cuda.synchronize()
-    barrier(world, dev)
-    ms_total = ev0.elapsed_time(ev1)
-    # per-kernel times: the same K steps again with the library's per-launch events
-    # (kept out of the main timed region: events between launches stop the next
-    # kernel's prologue from overlapping the previous kernel's tail)
-    opt.timing(True)
-    opt.timing_read()
-    for _ in range(args.steps):
-        opt.step(groups)
-    phases = opt.timing_read()
-    opt.timing(False)
-    t_load = time.perf_counter()
-    while time.perf_counter() - t_load < 0.4:
-        for _ in range(10):
-            opt.step(groups)
-        torch.cuda.synchronize()
-    clk = clocks.stop()
-    ms_total = max_over_ranks(ms_total, world, dev)
-    ms_step = ms_total / args.steps
+    # device-resident timed region, inside an untimed load window of 1 s
+    ms_step, burst_ms, phases, clk = measure(opt, groups, args.steps, args.warmup, world, dev, 1.0, local)
 
     flops_nom = w.ns_flops_nominal()
     value = flops_nom * world / (ms_step * 1e-3) / 1e12
     launches = sum(n for (_, n) in phases.values())
-    gemm_ms = sum(phases[k][0] for k in ("gram", "poly", "update")) / args.steps
-    ns_tflops = flops_nom / (gemm_ms * 1e-3) / 1e12
-    b_mom, b_app = elementwise_bytes(w)
-    mom_ms = phases["momentum_norm"][0] / max(phases["momentum_norm"][1], 1)
+    _, _, b_app = elementwise_bytes(w)
     apply_fused = phases["apply"][1] == 0
     app_ms = phases["apply"][0] / max(phases["apply"][1], 1)
     upd_ms = phases["update"][0] / max(phases["update"][1], 1)
@@ -368,6 +445,7 @@ def run_ours(args, w):
     # the timed region runs after >= 1 s of continuous load: the sustained bf16 peak
     # (measured under the power cap) is the denominator of the GEMM fractions
     tpeak = peaks["bf16_tflops_sustained"]
+    nsf = ns_figures(w, ms_step, burst_ms, phases, args.steps, peaks, world)
 
     # --- end to end through the host-buffer entry point (pinned host memory)
     Whp = [x.clone().pin_memory() for x in Wh]
@@ -375,6 +453,7 @@ def run_ours(args, w):
     Ghp = [x.clone().pin_memory() for x in Gh]
     hgroups = groups_of(w, Whp, Ghp, Bhp)
     e2e_steps = max(1, min(args.steps, 10))
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     opt.step_host(hgroups)
     opt.sync()
     barrier(world, dev)
@@ -403,11 +482,13 @@ def run_ours(args, w):
                            else "tcgen05 cta_group::1, 128x256 tiles",
                    "l2": f"working set {ws_bytes / 2**20:.0f} MiB > 126 MiB L2 (no flush)",
                    "flops_per_step_nominal": flops_nom, "flops_per_step_symmetric": w.ns_flops_symmetric()},
-        "ns5_tflops": round(ns_tflops, 2),
-        "ns5_frac_of_bf16_peak": round(ns_tflops / tpeak, 4),
-        "ns5_peak": f"{tpeak} TFLOP/s ({peak_src} sustained bf16 dense)",
-        "momentum_gbs": round(b_mom / (mom_ms * 1e-3) / 1e9, 1),
-        "momentum_frac_of_hbm": round(b_mom / (mom_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "value_basis": "nominal 5(4m^2n+2m^3) Newton-Schulz FLOPs x ranks / ms_per_step",
+        "ns5_peaks": {"sustained": peaks["bf16_tflops_sustained"], "burst": peaks["bf16_tflops"],
+                      "source": f"{peak_src} bf16 dense"},
+    }
+    line.update(nsf)
+    line.update({
+        "momentum_peak": f"{peaks['hbm_gbs']} GB/s ({peak_src} HBM copy)",
         "apply_gbs": None if apply_fused else round(b_app / (app_ms * 1e-3) / 1e9, 1),
         "apply_frac_of_hbm": None if apply_fused else round(b_app / (app_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
         "apply": "fused into the epilogue of the last update GEMM" if apply_fused else "apply_kernel",
@@ -425,13 +506,17 @@ def run_ours(args, w):
                   "note": "same K steps right after warm-up, before the power cap engages; clocks not sampled"},
         "gpu_launches": int(launches),
         "clocks": clk,
-    }
+    })
     line["roofline"]["traffic"] = update_gemm_traffic(w)
+    opt.close()
+    del W, G, B, groups, hgroups, Whp, Bhp, Ghp
+    torch.cuda.empty_cache()
+    if not args.no_per_workload:
+        line["per_workload"] = per_workload_rows(args, world, dev, peaks, local, w.key)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
         print(json.dumps(line), flush=True)
-    opt.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
@@ -446,6 +531,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="square4096", choices=sorted(wl.BY_KEY))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the rows of the other four workloads")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)          # at least 3 untimed warm-up steps
     w = wl.get(args.workload)

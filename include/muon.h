@@ -211,6 +211,16 @@ muon_status muon_last_norms(muon_handle* h, float* out, int cap, int* n_out, voi
  * `stream`.  Valid until the next step or orthogonalisation on the handle. */
 muon_status muon_last_update(muon_handle* h, int group, int index, float* dst, void* stream);
 
+/* RMS of the update that the last muon_step applied to each matrix,
+ * lr * |s| * sqrt(sum(O^2) / (rows * cols)) with the matrix's per-shape scale s
+ * (the "实践 checklist" of the Muon note asks for the update RMS to be logged; with
+ * MUON_SCALE_MATCH_RMS and a full-rank O it is close to lr * rms_target).  Computed
+ * on the device from the final iterate in a fixed summation order, then copied to
+ * `out` (host, `cap` floats; groups in order, matrices in order); synchronises the
+ * stream.  *n_out gets the number of matrices.  After muon_orthogonalize it reports
+ * lr * RMS(O) of that call's outputs. */
+muon_status muon_last_update_rms(muon_handle* h, float* out, int cap, int* n_out, void* stream);
+
 /* Per-phase device timing.  While enabled, every launch of the step is
  * bracketed by CUDA events recorded on the launching stream.  muon_timing_read
  * synchronises the stream, adds the elapsed times of all launches since the last
@@ -248,7 +258,14 @@ const char* muon_status_string(muon_status s);
  * loads the library holds until the process exits; a matrix of more than
  * MUON_NOALLOC_MAX_BLOCKS * 8192 elements is rejected with MUON_ERR_UNSUPPORTED.
  * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * (cudaGetSymbolAddress) and keeps it for the life of the process, so make that
+ * first call before any stream capture.  With the CUDA runtime's lazy module
+ * loading (the default since CUDA 12) that first call is also when the module is
+ * loaded and the 512 KiB are reserved on the device: make it a warm-up call while
+ * device memory is still available.  After cudaDeviceReset on a device the kept
+ * address is stale; do not use this entry point on that device again in the
+ * process.  B, U_out and norm_out are written, so none of them may overlap another
+ * buffer of the call (MUON_ERR_INVALID).
  * All calls share the one array, and each call overwrites the partial sums it
  * reads: calls whose work overlaps on the GPU (unordered streams) race and give
  * wrong norms.  err_msg (optional host buffer of err_cap bytes) receives a

@@ -73,6 +73,8 @@ _SIGNATURES = {
     "muon_sync": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "muon_last_norms": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_float), ctypes.c_int,
                                        ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]),
+    "muon_last_update_rms": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_float), ctypes.c_int,
+                                            ctypes.POINTER(ctypes.c_int), ctypes.c_void_p]),
     "muon_last_update": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p]),
     "muon_timing_enable": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_int]),
     "muon_timing_read": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int),
@@ -152,22 +154,27 @@ def _dtype_code(t) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def _check_tensors(ts, shape, on_cuda: bool, dtype=None):
+def _check_tensors(ts, shape, on_cuda: bool, dtype=None, device: Optional[int] = None):
     """Same shape, dense, on the expected device kind and, when given, of one dtype
-    (the library reads and writes these buffers as dense arrays of that type)."""
+    (the library reads and writes these buffers as dense arrays of that type) and on
+    CUDA device `device` (the kernels run on one device and take only its memory)."""
     for t in ts:
         if tuple(t.shape) != tuple(shape) or not t.is_contiguous():
             raise ValueError(f"expected contiguous tensors of shape {tuple(shape)}, got {tuple(t.shape)}")
         if t.is_cuda != on_cuda:
             raise ValueError("tensor on the wrong device kind")
+        if on_cuda and device is not None and t.device.index != device:
+            raise ValueError(f"tensor on cuda:{t.device.index}, expected cuda:{device}")
         if dtype is not None and t.dtype != dtype:
             raise ValueError(f"expected {dtype} tensors, got {t.dtype}")
 
 
-def _stream(stream) -> int:
+def _stream(stream, device: Optional[int] = None) -> int:
+    """The raw cudaStream_t: the given stream, else the current stream of `device`
+    (of the current device when None)."""
     import torch
     if stream is None:
-        return torch.cuda.current_stream().cuda_stream
+        return torch.cuda.current_stream(device).cuda_stream
     return stream if isinstance(stream, int) else stream.cuda_stream
 
 
@@ -194,9 +201,9 @@ class Muon:
         for i, g in enumerate(groups):
             import torch
             rows, cols = g.W[0].shape
-            _check_tensors(g.W, (rows, cols), on_cuda, torch.float32)
-            _check_tensors(g.G, (rows, cols), on_cuda, g.G[0].dtype)
-            _check_tensors(g.B, (rows, cols), on_cuda, torch.float32)
+            _check_tensors(g.W, (rows, cols), on_cuda, torch.float32, self.device)
+            _check_tensors(g.G, (rows, cols), on_cuda, g.G[0].dtype, self.device)
+            _check_tensors(g.B, (rows, cols), on_cuda, torch.float32, self.device)
             if not (len(g.W) == len(g.G) == len(g.B)):
                 raise ValueError("W, G and B lists differ in length")
             pw, pg, pb = _ptrs(g.W), _ptrs(g.G), _ptrs(g.B)
@@ -225,12 +232,12 @@ class Muon:
     def step(self, groups: List[Group], stream=None):
         arr, keep = self._groups(groups, True)
         self._shapes = [(arr[i].rows, arr[i].cols, arr[i].count) for i in range(len(groups))]
-        self._check(lib().muon_step(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream))), "muon_step")
+        self._check(lib().muon_step(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream, self.device))), "muon_step")
 
     def step_host(self, groups: List[Group], stream=None):
         arr, keep = self._groups(groups, False)
         self._shapes = [(arr[i].rows, arr[i].cols, arr[i].count) for i in range(len(groups))]
-        self._check(lib().muon_step_host(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream))), "muon_step_host")
+        self._check(lib().muon_step_host(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream, self.device))), "muon_step_host")
 
     def orthogonalize(self, groups, stream=None):
         """groups: list of (M_list, O_list); O = NS(M / (||M||_F + eps)), fp32 outputs."""
@@ -239,21 +246,24 @@ class Muon:
         for i, (Ms, Os) in enumerate(groups):
             import torch
             rows, cols = Ms[0].shape
-            _check_tensors(Ms, (rows, cols), True, Ms[0].dtype)
-            _check_tensors(Os, (rows, cols), True, torch.float32)
+            _check_tensors(Ms, (rows, cols), True, Ms[0].dtype, self.device)
+            _check_tensors(Os, (rows, cols), True, torch.float32, self.device)
             pm, po = _ptrs(Ms), _ptrs(Os)
             keep += [pm, po]
             arr[i] = _OrthoGroup(rows, cols, len(Ms), _dtype_code(Ms[0]),
                                  ctypes.cast(pm, ctypes.POINTER(ctypes.c_void_p)),
                                  ctypes.cast(po, ctypes.POINTER(ctypes.c_void_p)))
-        self._check(lib().muon_orthogonalize(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream))),
+        self._check(lib().muon_orthogonalize(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream, self.device))),
                     "muon_orthogonalize")
 
     def ns_phase(self, phase: int, precision: int, m: int, n: int, count: int, alpha: float, beta: float,
                  x_op=None, a_in=None, x_master=None, out=None, out_op=None, stream=None):
+        for t in (x_op, a_in, x_master, out, out_op):
+            if t is not None and (not t.is_cuda or t.device.index != self.device):
+                raise ValueError(f"building-block buffers must be on cuda:{self.device}")
         p = lambda t: None if t is None else t.data_ptr()
         args = _PhaseArgs(phase, precision, m, n, count, alpha, beta, p(x_op), p(a_in), p(x_master), p(out), p(out_op))
-        self._check(lib().muon_ns_phase_run(self._h, ctypes.byref(args), ctypes.c_void_p(_stream(stream))),
+        self._check(lib().muon_ns_phase_run(self._h, ctypes.byref(args), ctypes.c_void_p(_stream(stream, self.device))),
                     "muon_ns_phase_run")
 
     def qk_clip(self, Wq, Wk, max_logits, head_dim: int, tau: float, stream=None):
@@ -264,6 +274,8 @@ class Muon:
                 continue
             if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
                 raise ValueError(f"{name} must be a contiguous float32 CUDA tensor")
+            if t.device.index != self.device:
+                raise ValueError(f"{name} is on cuda:{t.device.index}, the handle on cuda:{self.device}")
         n_heads = max_logits.numel()
         if Wq.dim() != 2:
             raise ValueError("Wq must be 2-D")
@@ -273,17 +285,26 @@ class Muon:
         self._check(lib().muon_qk_clip(self._h, ctypes.c_void_p(Wq.data_ptr()),
                                        None if Wk is None else ctypes.c_void_p(Wk.data_ptr()),
                                        ctypes.c_void_p(max_logits.data_ptr()), n_heads, head_dim, cols, float(tau),
-                                       ctypes.c_void_p(_stream(stream))), "muon_qk_clip")
+                                       ctypes.c_void_p(_stream(stream, self.device))), "muon_qk_clip")
 
     def sync(self, stream=None):
-        self._check(lib().muon_sync(self._h, ctypes.c_void_p(_stream(stream))), "muon_sync")
+        self._check(lib().muon_sync(self._h, ctypes.c_void_p(_stream(stream, self.device))), "muon_sync")
 
     def last_norms(self, stream=None) -> List[float]:
         n = ctypes.c_int(0)
-        lib().muon_last_norms(self._h, None, 0, ctypes.byref(n), ctypes.c_void_p(_stream(stream)))
+        lib().muon_last_norms(self._h, None, 0, ctypes.byref(n), ctypes.c_void_p(_stream(stream, self.device)))
         buf = (ctypes.c_float * max(n.value, 1))()
-        self._check(lib().muon_last_norms(self._h, buf, n.value, ctypes.byref(n), ctypes.c_void_p(_stream(stream))),
+        self._check(lib().muon_last_norms(self._h, buf, n.value, ctypes.byref(n), ctypes.c_void_p(_stream(stream, self.device))),
                     "muon_last_norms")
+        return list(buf[: n.value])
+
+    def last_update_rms(self, stream=None) -> List[float]:
+        """Per matrix (groups in order), the RMS of the update lr * s * O of the last step."""
+        n = ctypes.c_int(0)
+        lib().muon_last_update_rms(self._h, None, 0, ctypes.byref(n), ctypes.c_void_p(_stream(stream, self.device)))
+        buf = (ctypes.c_float * max(n.value, 1))()
+        self._check(lib().muon_last_update_rms(self._h, buf, n.value, ctypes.byref(n),
+                                               ctypes.c_void_p(_stream(stream, self.device))), "muon_last_update_rms")
         return list(buf[: n.value])
 
     def last_update(self, group: int, index: int, dst, stream=None):
@@ -293,9 +314,9 @@ class Muon:
         shapes = getattr(self, "_shapes", None)
         if shapes is None or not (0 <= group < len(shapes)) or not (0 <= index < shapes[group][2]):
             raise ValueError(f"no matrix {index} in group {group} of the last call")
-        _check_tensors([dst], shapes[group][:2], True, torch.float32)
+        _check_tensors([dst], shapes[group][:2], True, torch.float32, self.device)
         self._check(lib().muon_last_update(self._h, group, index, ctypes.c_void_p(dst.data_ptr()),
-                                           ctypes.c_void_p(_stream(stream))), "muon_last_update")
+                                           ctypes.c_void_p(_stream(stream, self.device))), "muon_last_update")
 
     TIMING_KINDS = ("momentum_norm", "norm_finalize", "gram", "poly", "update", "apply")
 
@@ -307,7 +328,7 @@ class Muon:
         k = len(self.TIMING_KINDS)
         ms = (ctypes.c_double * k)()
         n = (ctypes.c_int * k)()
-        self._check(lib().muon_timing_read(self._h, ms, n, k, ctypes.c_void_p(_stream(stream))), "muon_timing_read")
+        self._check(lib().muon_timing_read(self._h, ms, n, k, ctypes.c_void_p(_stream(stream, self.device))), "muon_timing_read")
         return {name: (ms[i], n[i]) for i, name in enumerate(self.TIMING_KINDS)}
 
     def close(self):
@@ -327,16 +348,24 @@ def momentum_norm_noalloc(G, B, norm_out, U_out=None, momentum: float = 0.95, ne
     B <- momentum*B + G in place, U_out = G + momentum*B (or B), norm_out[0] = ||U||_F."""
     import torch
     rows, cols = B.shape
-    _check_tensors([G], (rows, cols), True)
-    _check_tensors([B], (rows, cols), True, torch.float32)
+    if not B.is_cuda:
+        raise ValueError("B must be a CUDA tensor")
+    dev = B.device.index
+    _check_tensors([G], (rows, cols), True, None, dev)
+    _check_tensors([B], (rows, cols), True, torch.float32, dev)
     if U_out is not None:
-        _check_tensors([U_out], (rows, cols), True, torch.float32)
+        _check_tensors([U_out], (rows, cols), True, torch.float32, dev)
     if norm_out.dtype != torch.float32 or not norm_out.is_cuda or norm_out.numel() < 1:
         raise ValueError("norm_out must be a float32 CUDA tensor with at least one element")
+    if norm_out.device.index != dev:
+        raise ValueError(f"norm_out is on cuda:{norm_out.device.index}, B on cuda:{dev}")
     err = ctypes.create_string_buffer(256)
-    st = lib().muon_momentum_norm_noalloc(rows, cols, _dtype_code(G), G.data_ptr(), B.data_ptr(),
-                                          None if U_out is None else U_out.data_ptr(), float(momentum), int(nesterov),
-                                          norm_out.data_ptr(), ctypes.c_void_p(_stream(stream)), err, 256)
+    # the entry point works on the current device: make it B's for the call
+    with torch.cuda.device(dev):
+        st = lib().muon_momentum_norm_noalloc(rows, cols, _dtype_code(G), G.data_ptr(), B.data_ptr(),
+                                              None if U_out is None else U_out.data_ptr(), float(momentum),
+                                              int(nesterov), norm_out.data_ptr(), ctypes.c_void_p(_stream(stream)),
+                                              err, 256)
     if st != MUON_OK:
         raise MuonError(st, f"muon_momentum_norm_noalloc: {err.value.decode()}")
 

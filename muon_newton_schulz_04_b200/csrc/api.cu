@@ -70,6 +70,8 @@ struct Plan {
     float* d_norms = nullptr;
     float* d_scale = nullptr;
     int* d_counters = nullptr;           // per-matrix block counters of the momentum kernel
+    double* d_rms_part = nullptr;        // update-RMS partial sums (UPDATE_RMS_PARTIALS per matrix)
+    float* d_rms = nullptr;              // update RMS per matrix
     bool valid = false;
     unsigned long long version = 0;      // distinct per built plan
     std::vector<EwSeg> uploaded;         // last segment table copied to the device
@@ -316,18 +318,32 @@ muon_status load_encoder(muon_handle* h) {
 // 3-D bf16 tensor map over [count][rows][ld] with the logical width `cols`:
 // box of box_cols (= 64, one 128-byte swizzle span) x box_rows, 128-byte swizzle,
 // zero fill outside.
-muon_status encode_map(muon_handle* h, CUtensorMap* m, const void* base, int cols, int rows, int count, int ld,
-                       int box_rows) {
+muon_status encode_map_box(muon_handle* h, CUtensorMap* m, const void* base, int cols, int rows, int count, int ld,
+                           int box_cols, int box_rows, CUtensorMapSwizzle swz) {
     cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, (cuuint64_t)count};
     cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)ld * 2 * (cuuint64_t)rows};
-    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+    cuuint32_t box[3] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = h->encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
-        return fail(h, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %dx%dx%d ld %d", (int)r, count, rows, cols, ld);
+        return fail(h, MUON_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %dx%dx%d ld %d box %dx%d", (int)r, count,
+                    rows, cols, ld, box_rows, box_cols);
     return MUON_OK;
+}
+
+muon_status encode_map(muon_handle* h, CUtensorMap* m, const void* base, int cols, int rows, int count, int ld,
+                       int box_rows) {
+    return encode_map_box(h, m, base, cols, rows, count, ld, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// 32-row boxes of the UPDATE epilogue (tc_gemm_epi_cols() columns, the swizzle whose
+// span is one box row).
+muon_status encode_epi_map(muon_handle* h, CUtensorMap* m, const void* base, int cols, int rows, int count, int ld) {
+    const int bc = tc_gemm_epi_cols();
+    return encode_map_box(h, m, base, cols, rows, count, ld, bc, 32,
+                          bc == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
 }
 
 bool is_bf16_path(const muon_handle* h) { return h->cfg.precision == MUON_PREC_BF16; }
@@ -433,6 +449,7 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
     const size_t o_segs = take(P.segs.size() * sizeof(EwSeg)), o_part = take((size_t)k1 * sizeof(double) + 8);
     const size_t o_norm = take((size_t)mat * sizeof(float)), o_scale = take((size_t)mat * sizeof(float));
     const size_t o_cnt = take((size_t)mat * sizeof(int));
+    const size_t o_rmsp = take((size_t)mat * UPDATE_RMS_PARTIALS * sizeof(double)), o_rms = take((size_t)mat * sizeof(float));
     size_t o_units[3], o_ubeg[3];
     for (int ph = 0; ph < 3; ++ph) {
         o_units[ph] = take(upl[ph].units.size() * 2 * sizeof(int4) + 32);
@@ -464,6 +481,8 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
     P.d_norms = reinterpret_cast<float*>(base + o_norm);
     P.d_scale = reinterpret_cast<float*>(base + o_scale);
     P.d_counters = reinterpret_cast<int*>(base + o_cnt);
+    P.d_rms_part = reinterpret_cast<double*>(base + o_rmsp);
+    P.d_rms = reinterpret_cast<float*>(base + o_rms);
     CUDA_TRY(h, cudaMemsetAsync(P.d_counters, 0, (size_t)mat * sizeof(int), s));
 
     // workspace pointers in the segment table
@@ -494,6 +513,10 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
             }
             if ((st = encode_map(h, &maps[g].a, base + o.a, d.m, d.m, d.count, d.ldm, 128)) != MUON_OK) return st;
             if ((st = encode_map(h, &maps[g].p, base + o.p, d.m, d.m, d.count, d.ldm, 128)) != MUON_OK) return st;
+            for (int b = 0; b < 2; ++b)
+                if ((st = encode_epi_map(h, &maps[g].xe_hi[b], base + o.xb[b], d.n, d.m, d.count, d.ldn)) != MUON_OK) return st;
+            if ((st = encode_epi_map(h, &maps[g].xe_lo_in, base + o.xl, d.n, d.m, d.count, d.ldn)) != MUON_OK) return st;
+            maps[g].xe_lo_out = maps[g].xe_lo_in;
             GemmGroupInfo& q = gi[g];
             q.m = d.m; q.n = d.n; q.ldm = d.ldm; q.ldn = d.ldn; q.count = d.count; q.mat_base = P.mat_base[g];
             q.xb[0] = reinterpret_cast<__nv_bfloat16*>(base + o.xb[0]);
@@ -999,6 +1022,10 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     } else {
         if ((st = encode_map(h, &maps.p, a->a_in, m, m, cnt, m, 128)) != MUON_OK) return st;
         if ((st = encode_map(h, &maps.xb_mn[0], a->x_op, n, m, cnt, n, 64)) != MUON_OK) return st;
+        if ((st = encode_epi_map(h, &maps.xe_hi[0], a->x_op, n, m, cnt, n)) != MUON_OK) return st;
+        if ((st = encode_epi_map(h, &maps.xe_hi[1], a->out, n, m, cnt, n)) != MUON_OK) return st;
+        if ((st = encode_epi_map(h, &maps.xe_lo_in, a->x_master, n, m, cnt, n)) != MUON_OK) return st;
+        if ((st = encode_epi_map(h, &maps.xe_lo_out, a->out_op, n, m, cnt, n)) != MUON_OK) return st;
         gi.xb[0] = (__nv_bfloat16*)a->x_op;            // X = x_op + x_master (high + low part)
         gi.xlo_in = (const __nv_bfloat16*)a->x_master;
         gi.xb[1] = (__nv_bfloat16*)a->out;              // X' = out + out_op
@@ -1099,6 +1126,21 @@ muon_status muon_last_norms(muon_handle* h, float* out, int cap, int* n_out, voi
     DeviceGuard dg(h->device);
     CUDA_TRY(h, cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
     CUDA_TRY(h, cudaMemcpy(out, h->plan.d_norms, h->plan.nmat * sizeof(float), cudaMemcpyDeviceToHost));
+    return MUON_OK;
+}
+
+muon_status muon_last_update_rms(muon_handle* h, float* out, int cap, int* n_out, void* stream) {
+    if (!h || !n_out) return MUON_ERR_INVALID;
+    Plan& P = h->plan;
+    if (!P.valid || P.uploaded.empty()) return fail(h, MUON_ERR_INVALID, "no step has run on this handle");
+    *n_out = P.nmat;
+    if (!out || cap < P.nmat) return fail(h, MUON_ERR_INVALID, "output holds %d floats, %d needed", cap, P.nmat);
+    DeviceGuard dg(h->device);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    CUDA_TRY(h, launch_update_rms(P.d_segs, P.nmat, h->cfg.ns_steps == 0 ? P.d_scale : nullptr, h->cfg.lr,
+                                  P.d_rms_part, P.d_rms, s));
+    CUDA_TRY(h, cudaStreamSynchronize(s));
+    CUDA_TRY(h, cudaMemcpy(out, P.d_rms, P.nmat * sizeof(float), cudaMemcpyDeviceToHost));
     return MUON_OK;
 }
 

@@ -400,7 +400,57 @@ __global__ void __launch_bounds__(EW_THREADS) copy_out_one_kernel(const EwSeg sg
     apply_block(sg, blockIdx.x, 1.0f, 0.0f, o_scale, 1, dst);
 }
 
+// RMS of the applied update lr * s * O of every matrix, over the final iterate
+// (RMS does not depend on the orientation).  Block (c, mat) sums the squares of
+// rows c, c + RMS_CHUNKS, ... of the matrix's oriented m x n iterate in fp64;
+// update_rms_finish_kernel adds the RMS_CHUNKS partials of each matrix in a fixed
+// order, so the result is bitwise reproducible.
+constexpr int RMS_CHUNKS = 32;
+
+__global__ void __launch_bounds__(EW_THREADS) update_sq_kernel(const EwSeg* __restrict__ segs,
+                                                               const float* __restrict__ o_scale,
+                                                               double* __restrict__ part) {
+    __shared__ double red[EW_THREADS / 32];
+    pdl_trigger();
+    pdl_wait();
+    const EwSeg sg = segs[blockIdx.y];
+    const int m = sg.transposed ? sg.cols : sg.rows, n = sg.transposed ? sg.rows : sg.cols;
+    const float os = o_scale ? o_scale[sg.mat] : 1.0f;
+    double acc = 0.0;
+    for (int r = blockIdx.x; r < m; r += RMS_CHUNKS) {
+        for (int c = threadIdx.x; c < n; c += EW_THREADS) {
+            const double v = (double)(load_o(sg, (size_t)r * sg.ldn + c) * os);
+            acc += v * v;
+        }
+    }
+    const double tot = block_sum(acc, red);
+    if (threadIdx.x == 0) part[(size_t)blockIdx.y * RMS_CHUNKS + blockIdx.x] = tot;
+}
+
+__global__ void __launch_bounds__(32) update_rms_finish_kernel(const EwSeg* __restrict__ segs,
+                                                               const double* __restrict__ part, float lr,
+                                                               float* __restrict__ rms) {
+    pdl_trigger();
+    pdl_wait();
+    const EwSeg sg = segs[blockIdx.x];
+    double v = part[(size_t)blockIdx.x * RMS_CHUNKS + threadIdx.x];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0)
+        rms[blockIdx.x] = (float)((double)lr * fabs((double)sg.update_scale) *
+                                  sqrt(v / ((double)sg.rows * (double)sg.cols)));
+}
+static_assert(RMS_CHUNKS == 32, "the finish kernel reduces one warp");
+
 }  // namespace
+
+cudaError_t launch_update_rms(const EwSeg* segs, int nseg, const float* o_scale, float lr, double* part, float* rms,
+                              cudaStream_t s) {
+    if (nseg <= 0) return cudaSuccess;
+    cudaError_t e = launch_pdl(update_sq_kernel, dim3(RMS_CHUNKS, nseg), dim3(EW_THREADS), 0, s, segs, o_scale, part);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(update_rms_finish_kernel, dim3(nseg), dim3(32), 0, s, segs, (const double*)part, lr, rms);
+}
 
 cudaError_t launch_momentum_norm(const EwSeg* segs, int nseg, int nblocks, double* partials, float mu,
                                  int nesterov, int bf16_operand, int* counters, float eps, float* norms,

@@ -63,8 +63,46 @@ constexpr int S1_SMEM = 1024 + S1_STAGES * (S1_A + S1_B) + 256 + STAGE_BYTES;
 constexpr int S2_BM = 256, S2_BN = 256, S2_STAGES = MUON_S2_STAGES;
 constexpr int S2_A = 128 * BK * 2;            // 16 KiB: this CTA's 128 rows of A
 constexpr int S2_B = 128 * BK * 2;            // 16 KiB: this CTA's 128 columns of B
-constexpr int S2_SMEM = 1024 + S2_STAGES * (S2_A + S2_B) + 256 + STAGE_BYTES;
-static_assert(S1_SMEM <= 232448 && S2_SMEM <= 232448, "dynamic shared memory above the 227 KiB limit");
+
+// UPDATE epilogue of the two-CTA kernel: each epilogue warp streams its 32 rows of
+// the iterate through a private ring of EU_DEPTH shared-memory buffers, one
+// 32-row x EU_COLS-column box of hi and one of lo per buffer, loaded by TMA up to
+// EU_DEPTH - 1 chunks ahead (across tile boundaries) and written back in place, then
+// stored by TMA.  The operand ring of this mode is S2U_STAGES deep.
+#ifndef MUON_EU_COLS
+#define MUON_EU_COLS 32
+#endif
+#ifndef MUON_EU_DEPTH
+#define MUON_EU_DEPTH 3
+#endif
+#ifndef MUON_S2U_STAGES
+#define MUON_S2U_STAGES 4
+#endif
+constexpr int EU_COLS = MUON_EU_COLS;               // 16 or 32 columns per chunk
+constexpr int EU_DEPTH = MUON_EU_DEPTH;
+constexpr int EU_ROW_BYTES = EU_COLS * 2;           // one bf16 row of a box: 32 or 64 bytes
+constexpr int EU_BOX = 32 * EU_ROW_BYTES;           // one 32-row box
+constexpr int EU_BUF = 2 * EU_BOX;                  // hi + lo
+constexpr int S2U_STAGES = MUON_S2U_STAGES;
+static_assert(EU_COLS == 16 || EU_COLS == 32, "epilogue chunks are 16 or 32 columns");
+static_assert(EU_DEPTH >= 2 && EU_DEPTH <= 8, "epilogue ring depth out of range");
+
+constexpr int s2_stages(int mode) { return mode == MODE_UPDATE ? S2U_STAGES : S2_STAGES; }
+constexpr int s2_epi_bytes(int mode) { return mode == MODE_UPDATE ? NUM_EPI_WARPS * EU_DEPTH * EU_BUF : STAGE_BYTES; }
+// barriers: full / empty per stage, two tfull / tempty, drain, the epilogue ring's
+// (UPDATE), then the TMEM address and the abort flag
+constexpr int s2_bar_bytes(int mode) {
+    return (8 * (2 * s2_stages(mode) + 5 + (mode == MODE_UPDATE ? NUM_EPI_WARPS * EU_DEPTH : 0)) + 8 + 127) / 128 * 128;
+}
+// [operand ring][epilogue buffers][barriers]; the ring and the buffers are 1024-byte aligned
+constexpr int s2_smem(int mode) {
+    return 1024 + s2_stages(mode) * (S2_A + S2_B) + s2_epi_bytes(mode) + s2_bar_bytes(mode);
+}
+constexpr int S2_SMEM = s2_smem(MODE_GRAM);
+constexpr int S2U_SMEM = s2_smem(MODE_UPDATE);
+static_assert(S1_SMEM <= 232448 && S2_SMEM <= 232448 && S2U_SMEM <= 232448,
+              "dynamic shared memory above the 227 KiB limit");
+static_assert((s2_stages(MODE_UPDATE) * (S2_A + S2_B)) % 1024 == 0 && EU_BUF % 1024 == 0, "buffer alignment");
 
 // error codes written to the device error word when a bounded wait gives up
 constexpr int ERR_PRODUCER = 0x101, ERR_MMA_SLOT = 0x102, ERR_MMA_ACC = 0x103, ERR_EPILOGUE = 0x104,
@@ -483,6 +521,102 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
     while (globaltimer_ns() - t0 < ns) { }
 }
 
+// 32 lanes x 16 columns of 32-bit accumulators (lane i: row base_lane + i).
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+        " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
+
+template <int NC>
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&r)[NC]) {
+    if constexpr (NC == 32) tmem_ld_32x32b_x32(taddr, r);
+    else tmem_ld_32x32b_x16(taddr, r);
+}
+
+// Weight update (apply_mode 1) or copy-out (apply_mode 2) of NC finished values
+// O[row][col0 .. col0 + NC) of the oriented result, one row per lane.  A matrix that
+// was transposed for the smaller Gram gets W[c][row]: lanes hold consecutive rows,
+// so each store instruction of the warp covers 32 consecutive elements of W's row c.
+template <int NC>
+__device__ __forceinline__ void apply_row(const GemmParams& p, const GemmGroupInfo& gi, const EwSeg& sg, int row,
+                                          int col0, const float (&val)[NC]) {
+    float* w = sg.w;
+    const float step = p.lr * sg.update_scale;
+    const bool copy = p.apply_mode == 2;
+    if (!sg.transposed) {
+        float* wr = w + (size_t)row * sg.cols;
+        if (sg.vec && col0 + NC - 1 < gi.n) {
+            float4* w4 = reinterpret_cast<float4*>(wr + col0);
+#pragma unroll
+            for (int qq = 0; qq < NC / 4; ++qq) {
+                float4 o = make_float4(val[4 * qq], val[4 * qq + 1], val[4 * qq + 2], val[4 * qq + 3]);
+                if (!copy) {
+                    const float4 x = w4[qq];
+                    o.x = fmaf(-step, o.x, p.decay * x.x);
+                    o.y = fmaf(-step, o.y, p.decay * x.y);
+                    o.z = fmaf(-step, o.z, p.decay * x.z);
+                    o.w = fmaf(-step, o.w, p.decay * x.w);
+                }
+                w4[qq] = o;
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < NC; ++j) {
+                const int c = col0 + j;
+                if (c < gi.n) wr[c] = copy ? val[j] : fmaf(-step, val[j], p.decay * wr[c]);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < NC; ++j) {
+            const int c = col0 + j;
+            if (c < gi.n) {
+                float* wp = w + (size_t)c * sg.cols + row;
+                *wp = copy ? val[j] : fmaf(-step, val[j], p.decay * *wp);
+            }
+        }
+    }
+}
+
+// Where chunk c of unit u lies for one epilogue warp of the two-CTA UPDATE kernel:
+// the warp's 32 rows (CTA `rank`, TMEM lane quarter q) and EU_COLS columns of its
+// column half.  A chunk is a "load chunk" when it needs the iterate (its unit is not
+// a split part that only stores a partial sum) and touches the matrix.
+struct EuChunk {
+    int g, mat, row0, col0, tcol;   // group, matrix, first row / column, TMEM column
+    bool load;
+};
+
+__device__ __forceinline__ int eu_nchunks(int4 sk) {
+    return (sk.z & 0xFF) == 2 ? 0 : ((sk.z >> 8) ? 64 : 128) / EU_COLS;
+}
+
+__device__ __forceinline__ EuChunk eu_chunk(const GemmParams& p, int4 tile, int4 sk, int c, int rank, int q,
+                                            int half) {
+    const int nh = sk.z >> 8;
+    EuChunk ch;
+    ch.g = tile.x;
+    ch.mat = tile.y;
+    ch.row0 = tile.z * S2_BM + rank * 128 + q * 32;
+    ch.tcol = half * (nh ? 64 : 128) + c * EU_COLS;
+    ch.col0 = tile.w * S2_BN + (nh ? (nh - 1) * 128 : 0) + ch.tcol;
+    const GemmGroupInfo& gi = p.groups[tile.x];
+    ch.load = (sk.z & 0xFF) != 2 && ch.row0 < gi.m && ch.col0 < gi.n;
+    return ch;
+}
+
+// Byte offset of 16-byte slot k of row r inside a TMA box with EU_ROW_BYTES-byte rows
+// and the matching swizzle (64B: slot ^= (r >> 1) & 3; 32B: slot ^= (r >> 2) & 1).
+__device__ __forceinline__ uint32_t eu_off(int r, int k) {
+    constexpr int NS = EU_ROW_BYTES / 16;
+    constexpr int SH = EU_ROW_BYTES == 64 ? 1 : 2;
+    return (uint32_t)(r * EU_ROW_BYTES + ((k ^ ((r >> SH) & (NS - 1))) << 4));
+}
+
 // ============================================================================ one-CTA kernel
 
 template <int MODE>
@@ -644,21 +778,215 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ns_gemm_tc_kernel(const __grid
     }
 }
 
+// ============================================================================ two-CTA UPDATE epilogue
+
+// L2 prefetch of the weight elements that the fused apply of this thread's row will
+// read and write (apply_mode 1 only); the iterate itself arrives by TMA.
+__device__ __forceinline__ void prefetch_w_row(const GemmParams& p, const GemmGroupInfo& gi, int mat, int row,
+                                               int col_start, int ncols) {
+    if (p.apply_mode != 1 || row >= gi.m || col_start >= gi.n) return;
+    const EwSeg& sg = p.segs[gi.mat_base + mat];
+    const int ncw = min(ncols, gi.n - col_start);
+    if (!sg.transposed) {
+        const float* wr = sg.w + (size_t)row * sg.cols + col_start;
+        if (sg.vec) prefetch_l2_bulk(wr, (uint32_t)ncw * 4u);
+        else for (int c = 0; c < ncw; c += 32) prefetch_l2_line(wr + c);
+    } else {
+        const int lane = (int)(threadIdx.x & 31u);
+        const int row0 = row - lane;
+        for (int c = lane; c < ncw; c += 32) prefetch_l2_line(sg.w + (size_t)(col_start + c) * sg.cols + row0);
+    }
+}
+
+// One epilogue warp of the two-CTA UPDATE kernel: X' = alpha * acc + beta * (hi + lo),
+// stored as the pair hi' = bf16(X'), lo' = bf16(X' - hi'), for the warp's 32 rows of
+// every unit of its cluster, chunk by chunk (EU_COLS columns).  Lane 0 keeps up to
+// EU_DEPTH - 1 chunks of the iterate in flight: TMA loads of the hi and lo boxes into
+// the warp's ring buffer, completing on the buffer's mbarrier.  Each lane owns one
+// row (the tcgen05.ld 32x32b layout) and reads and rewrites its row of both boxes in
+// place (swizzled, bank-conflict free); lane 0 then stores the boxes by TMA, waits
+// until the previous chunk's stores have read their buffer and reuses it for the next
+// load.  Returns false when a bounded wait gave up.
+__device__ __forceinline__ bool update_epilogue_pair(const GemmParams& p, uint32_t rank, uint32_t warp,
+                                                  uint32_t tmem_base, uint8_t* ebuf, uint64_t* ebar,
+                                                  uint64_t* tfull, uint64_t* tempty, volatile int* abort_flag,
+                                                  int cid) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const int q = (int)(warp & 3u), half = (int)((warp - 2) >> 2);
+    const int u_begin = p.unit_begin[cid], u_end = p.unit_begin[cid + 1];
+    // issuer (lane 0): the next (unit, chunk) to look at and the loads issued so far
+    int iu = u_begin, ic = 0;
+    uint32_t issued = 0, consumed = 0;
+    auto issue_next = [&]() {
+        while (iu < u_end) {
+            const int4 tile = p.units[2 * iu], sk = p.units[2 * iu + 1];
+            if (ic >= eu_nchunks(sk)) { ++iu; ic = 0; continue; }
+            const EuChunk ch = eu_chunk(p, tile, sk, ic, (int)rank, q, half);
+            ++ic;
+            if (!ch.load) continue;
+            const uint32_t b = issued % EU_DEPTH;
+            uint8_t* dst = ebuf + b * EU_BUF;
+            const GemmMaps& mp = p.maps[ch.g];
+            mbar_arrive_expect_tx(&ebar[b], EU_BUF);
+            tma_load_3d(dst, &mp.xe_hi[p.parity], &ebar[b], ch.col0, ch.row0, ch.mat);
+            tma_load_3d(dst + EU_BOX, &mp.xe_lo_in, &ebar[b], ch.col0, ch.row0, ch.mat);
+            ++issued;
+            return;
+        }
+    };
+    if (lane == 0)
+        for (int i = 0; i < EU_DEPTH - 1; ++i) issue_next();
+
+    bool ok = true;
+    int local = 0;
+    for (int u = u_begin; u < u_end && ok; ++u, ++local) {
+        const int4 tile = p.units[2 * u];
+        const int4 sk = p.units[2 * u + 1];
+        const int kind = sk.z & 0xFF, nh = sk.z >> 8, slot = sk.w & 0xFFFF, nsl = sk.w >> 16;
+        const GemmGroupInfo& gi = p.groups[tile.x];
+        const uint32_t acc = local & 1;
+        const uint32_t acc_phase = (local >> 1) & 1;
+        const int row_local = q * 32 + (int)lane;
+        const int row = tile.z * S2_BM + (int)rank * 128 + row_local;
+        if (kind != 2)
+            prefetch_w_row(p, gi, tile.y, row, tile.w * S2_BN + (nh ? (nh - 1) * 128 + half * 64 : half * 128),
+                           nh ? 64 : 128);
+        ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, ERR_EPILOGUE);
+        if (kind == 1 && lane == 0) {
+            for (int sl = 0; sl < nsl && ok; ++sl)
+                ok = flag_wait(&p.sk_flag[slot + sl], p.epoch, abort_flag, p.err, ERR_SPLIT);
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
+        if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+        tc_fence_after();
+        float alpha = p.alpha, beta = p.beta;
+        if (p.scale != nullptr) {
+            const float sc = p.scale[gi.mat_base + tile.y];
+            alpha *= sc;
+            beta *= sc;
+        }
+        float* sk_row = kind == 0 ? nullptr
+                      : p.sk_partial + (size_t)slot * SK_SLOT_FLOATS + ((size_t)rank * 128 + row_local) * 256;
+        const uint32_t tacc = tmem_base + acc * ACC_COLS + (((uint32_t)q * 32u) << 16);
+        const EwSeg* sg = p.apply_mode != 0 ? &p.segs[gi.mat_base + tile.y] : nullptr;
+        const int nch = (nh ? 64 : 128) / EU_COLS;
+        for (int c = 0; c < nch; ++c) {
+            const EuChunk ch = eu_chunk(p, tile, sk, c, (int)rank, q, half);
+            if (kind == 2) {
+                // a later K range of a split tile: its raw partial sum goes to the slot
+                uint32_t v[EU_COLS];
+                tmem_ld_row<EU_COLS>(tacc + (uint32_t)ch.tcol, v);
+                tmem_ld_wait();
+                float4* dst = reinterpret_cast<float4*>(sk_row + ch.tcol);
+#pragma unroll
+                for (int qq = 0; qq < EU_COLS / 4; ++qq)
+                    dst[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
+                                          __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
+                continue;
+            }
+            if (!ch.load) continue;               // the warp's rows or columns lie outside the matrix
+            uint32_t v[EU_COLS];
+            tmem_ld_row<EU_COLS>(tacc + (uint32_t)ch.tcol, v);
+            tmem_ld_wait();
+            if (kind == 1) {
+                for (int sl = 0; sl < nsl; ++sl) {
+                    const float4* src = reinterpret_cast<const float4*>(sk_row + (size_t)sl * SK_SLOT_FLOATS + ch.tcol);
+#pragma unroll
+                    for (int qq = 0; qq < EU_COLS / 4; ++qq) {
+                        const float4 x = __ldcg(src + qq);
+                        v[4 * qq + 0] = __float_as_uint(__uint_as_float(v[4 * qq + 0]) + x.x);
+                        v[4 * qq + 1] = __float_as_uint(__uint_as_float(v[4 * qq + 1]) + x.y);
+                        v[4 * qq + 2] = __float_as_uint(__uint_as_float(v[4 * qq + 2]) + x.z);
+                        v[4 * qq + 3] = __float_as_uint(__uint_as_float(v[4 * qq + 3]) + x.w);
+                    }
+                }
+            }
+            const uint32_t b = consumed % EU_DEPTH;
+            ok = mbar_wait(&ebar[b], (consumed / EU_DEPTH) & 1u, abort_flag, p.err, ERR_EPILOGUE);
+            if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
+            const uint32_t hi_s = smem_u32(ebuf + b * EU_BUF), lo_s = hi_s + EU_BOX;
+            float res[EU_COLS];
+#pragma unroll
+            for (int k = 0; k < EU_COLS / 8; ++k) {
+                const uint32_t off = eu_off((int)lane, k);
+                const uint4 hv = lds128(hi_s + off), lv = lds128(lo_s + off);
+                const uint32_t h4[4] = {hv.x, hv.y, hv.z, hv.w};
+                const uint32_t l4[4] = {lv.x, lv.y, lv.z, lv.w};
+                uint32_t ho[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = bf16_bits_lo(h4[e]) + bf16_bits_lo(l4[e]);
+                    const float x1 = bf16_bits_hi(h4[e]) + bf16_bits_hi(l4[e]);
+                    const float y0 = alpha * __uint_as_float(v[8 * k + 2 * e]) + beta * x0;
+                    const float y1 = alpha * __uint_as_float(v[8 * k + 2 * e + 1]) + beta * x1;
+                    const __nv_bfloat162 hh = __floats2bfloat162_rn(y0, y1);
+                    const float2 hf = __bfloat1622float2(hh);
+                    const __nv_bfloat162 ll = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
+                    ho[e] = *reinterpret_cast<const uint32_t*>(&hh);
+                    lo[e] = *reinterpret_cast<const uint32_t*>(&ll);
+                    // the stored pair is the result: the weight update uses exactly it
+                    res[8 * k + 2 * e] = bf16_bits_lo(ho[e]) + bf16_bits_lo(lo[e]);
+                    res[8 * k + 2 * e + 1] = bf16_bits_hi(ho[e]) + bf16_bits_hi(lo[e]);
+                }
+                sts128(hi_s + off, make_uint4(ho[0], ho[1], ho[2], ho[3]));
+                sts128(lo_s + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                const GemmMaps& mp = p.maps[ch.g];
+                tma_store_3d(&mp.xe_hi[p.parity ^ 1], ebuf + b * EU_BUF, ch.col0, ch.row0, ch.mat);
+                tma_store_3d(&mp.xe_lo_out, ebuf + b * EU_BUF + EU_BOX, ch.col0, ch.row0, ch.mat);
+                bulk_commit();
+                bulk_wait_read<1>();          // the previous chunk's buffer is free again
+                issue_next();
+            }
+            ++consumed;
+            if (sg != nullptr && row < gi.m) apply_row<EU_COLS>(p, gi, *sg, row, ch.col0, res);
+        }
+        if (!ok) break;
+        tc_fence_before();
+        if (kind == 2) __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+            if (kind == 2 && atomicAdd(&p.sk_count[slot], 1) == 2 * NUM_EPI_WARPS - 1) {
+                // last of the 16 epilogue warps of the pair: the slot is complete
+                p.sk_count[slot] = 0;
+                __threadfence();
+                st_release_gpu(&p.sk_flag[slot], p.epoch);
+            }
+            mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
+        }
+    }
+    if (lane == 0) {
+        bulk_wait_all();
+        // loads still in flight (after an abort) must land before the CTA retires
+        const uint64_t t0 = globaltimer_ns();
+        for (uint32_t i = consumed; i < issued; ++i)
+            while (!mbar_try_wait(&ebar[i % EU_DEPTH], (i / EU_DEPTH) & 1u) && globaltimer_ns() - t0 < 100000000ull) { }
+    }
+    __syncwarp();
+    return ok;
+}
+
 // ============================================================================ two-CTA kernel
 
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
 ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
+    constexpr int STAGES = s2_stages(MODE);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + S2_STAGES * S2_A;
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S2_STAGES * (S2_A + S2_B));
-    uint64_t* empty = full + S2_STAGES;
-    uint64_t* tfull = empty + S2_STAGES;
+    uint8_t* sB = smem + STAGES * S2_A;
+    uint8_t* sE = smem + STAGES * (S2_A + S2_B);          // epilogue buffers
+    uint64_t* full = reinterpret_cast<uint64_t*>(sE + s2_epi_bytes(MODE));
+    uint64_t* empty = full + STAGES;
+    uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* ebar = drain + 1;                            // UPDATE: EU_DEPTH per epilogue warp
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + (MODE == MODE_UPDATE ? NUM_EPI_WARPS * EU_DEPTH : 0));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const uint32_t warp = warp_id();
@@ -667,7 +995,7 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
     const int cid = (int)cluster_id_x();               // index of this pair's unit list
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < S2_STAGES; ++s) {
+        for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);                   // used in CTA 0: its producer's arrive + both CTAs' bytes
             mbar_init(&empty[s], 1);                  // one commit from the MMA thread
         }
@@ -676,6 +1004,8 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
             mbar_init(&tempty[b], 2 * NUM_EPI_WARPS); // used in CTA 0: epilogue warps of both CTAs
         }
         mbar_init(drain, 1);
+        if (MODE == MODE_UPDATE)
+            for (int i = 0; i < NUM_EPI_WARPS * EU_DEPTH; ++i) mbar_init(&ebar[i], 1);
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -718,12 +1048,12 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
                     } else {
                         tma_load_3d_pair(b_dst, mapB, full0, k0, colh, mat);
                     }
-                    if (++stage == S2_STAGES) { stage = 0; phase ^= 1u; }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
             }
-            for (int i = 0; i < S2_STAGES && ok; ++i) {
+            for (int i = 0; i < STAGES && ok; ++i) {
                 if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, ERR_TAIL)) ok = false;
-                if (++stage == S2_STAGES) { stage = 0; phase ^= 1u; }
+                if (++stage == STAGES) { stage = 0; phase ^= 1u; }
             }
             if (!ok || *abort_flag) spin_ns(2000000ull);
         }
@@ -760,7 +1090,7 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
                     const uint32_t e_peer = mapa_shared(smem_u32(&empty[stage]), 1);
                     tc_commit_pair(e_own);
                     tc_commit_pair(e_peer);
-                    if (++stage == S2_STAGES) { stage = 0; phase ^= 1u; }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
                 }
                 if (!ok) break;
                 tc_commit_pair(mapa_shared(smem_u32(&tfull[acc]), 0));
@@ -772,10 +1102,13 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
                 while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 100000000ull) { }
             }
         }
+    } else if (MODE == MODE_UPDATE) {
+        update_epilogue_pair(p, rank, warp, tmem_base, sE + (warp - 2) * (EU_DEPTH * EU_BUF),
+                             ebar + (warp - 2) * EU_DEPTH, tfull, tempty, abort_flag, cid);
     } else {
         const uint32_t q = warp & 3u;
         const uint32_t half = (warp - 2) >> 2;
-        float* stage = reinterpret_cast<float*>(smem + S2_STAGES * (S2_A + S2_B) + 256) + (warp - 2) * STAGE_FLOATS;
+        float* stage = reinterpret_cast<float*>(sE) + (warp - 2) * STAGE_FLOATS;
         int local = 0;
         const int u_end = p.unit_begin[cid + 1];
         for (int u = p.unit_begin[cid]; u < u_end; ++u, ++local) {
@@ -832,6 +1165,8 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
 }  // namespace
 
 size_t tc_gemm_smem_bytes(int pair) { return pair ? S2_SMEM : S1_SMEM; }
+size_t tc_gemm_smem_bytes_mode(int mode, int pair) { return pair ? (size_t)s2_smem(mode) : (size_t)S1_SMEM; }
+int tc_gemm_epi_cols() { return EU_COLS; }
 int tc_gemm_threads() { return NUM_THREADS; }
 int tc_gemm_tile_m(int pair) { return pair ? S2_BM : S1_BM; }
 int tc_gemm_tile_n(int pair) { return pair ? S2_BN : S1_BN; }
@@ -843,7 +1178,7 @@ cudaError_t tc_gemm_prepare() {
     if ((e = cudaFuncSetAttribute(ns_gemm_tc_kernel<MODE_UPDATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, S1_SMEM)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_GRAM>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM)) != cudaSuccess) return e;
-    return cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_UPDATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM);
+    return cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_UPDATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2U_SMEM);
 }
 
 cudaError_t tc_gemm_max_clusters(int* n) {
@@ -855,10 +1190,16 @@ cudaError_t tc_gemm_max_clusters(int* n) {
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2, 1, 1);
     cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = S2_SMEM;
+    cfg.dynamicSmemBytes = S2U_SMEM;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaOccupancyMaxActiveClusters(n, ns_gemm_tc2_kernel<MODE_UPDATE>, &cfg);
+    int nu = 0, ng = 0;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&nu, ns_gemm_tc2_kernel<MODE_UPDATE>, &cfg);
+    if (e != cudaSuccess) return e;
+    cfg.dynamicSmemBytes = S2_SMEM;
+    e = cudaOccupancyMaxActiveClusters(&ng, ns_gemm_tc2_kernel<MODE_GRAM>, &cfg);
+    *n = nu < ng ? nu : ng;
+    return e;
 }
 
 cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cudaStream_t s) {
@@ -868,7 +1209,7 @@ cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cu
         switch (mode) {
             case MODE_GRAM: return launch_pdl(ns_gemm_tc2_kernel<MODE_GRAM>, g, b, S2_SMEM, s, p);
             case MODE_POLY: return launch_pdl(ns_gemm_tc2_kernel<MODE_POLY>, g, b, S2_SMEM, s, p);
-            default: return launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE>, g, b, S2_SMEM, s, p);
+            default: return launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE>, g, b, S2U_SMEM, s, p);
         }
     }
     switch (mode) {

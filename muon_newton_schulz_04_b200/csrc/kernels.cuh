@@ -57,6 +57,12 @@ struct alignas(64) GemmMaps {
     CUtensorMap xb_mn[2];  // X operand, box {64, 64}: X as an N-contiguous operand
     CUtensorMap a;         // A, box {64, 128}
     CUtensorMap p;         // P, box {64, 128}
+    // UPDATE epilogue of the two-CTA kernel: 32 x 32 boxes of the iterate, 64-byte
+    // swizzle, loaded into and stored from shared memory (hi in / hi out follow the
+    // ping-pong parity; lo in and lo out are the same array in a step)
+    CUtensorMap xe_hi[2];
+    CUtensorMap xe_lo_in;
+    CUtensorMap xe_lo_out;
 };
 
 struct GemmGroupInfo {
@@ -101,6 +107,9 @@ constexpr int SK_SLOT_FLOATS = 2 * 128 * 256;
 // pair = 1: the two-CTA kernel (256 x 256 tiles, grid = 2 x clusters);
 // pair = 0: the one-CTA kernel (128 x 256 tiles).
 size_t tc_gemm_smem_bytes(int pair);
+size_t tc_gemm_smem_bytes_mode(int mode, int pair);
+// columns of one box of the two-CTA UPDATE epilogue (16 or 32; boxes are 32 rows)
+int tc_gemm_epi_cols();
 int tc_gemm_threads();
 int tc_gemm_tile_m(int pair);
 int tc_gemm_tile_n(int pair);
@@ -134,6 +143,11 @@ cudaError_t launch_momentum_norm(const EwSeg* segs, int nseg, int nblocks, doubl
 cudaError_t launch_apply(const EwSeg* segs, int nseg, int nblocks, float decay, float lr,
                          const float* o_scale, int copy_out, cudaStream_t s);
 cudaError_t launch_copy_out_one(const EwSeg& seg, float* dst, const float* o_scale, cudaStream_t s);
+// Per matrix: rms[i] = lr * |s_i| * sqrt(sum of O_i^2 / (rows * cols)) over the final
+// iterate; `part` holds 32 doubles per matrix (fixed-order partial sums).
+constexpr int UPDATE_RMS_PARTIALS = 32;
+cudaError_t launch_update_rms(const EwSeg* segs, int nseg, const float* o_scale, float lr, double* part, float* rms,
+                              cudaStream_t s);
 // QK-Clip: rows of head h of W_q and W_k (n_heads * head_dim rows, `cols` columns)
 // times sqrt(min(1, tau / max_logits[h])).  wk may be nullptr.
 cudaError_t launch_qk_clip(float* wq, float* wk, const float* max_logits, int n_heads, int head_dim, int cols,

@@ -83,6 +83,12 @@ void put_msg(char* buf, int cap, const char* msg) {
     if (buf && cap > 0) snprintf(buf, (size_t)cap, "%s", msg);
 }
 
+// [a, a + na) and [b, b + nb) share at least one byte.
+bool spans_overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
 }  // namespace
 }  // namespace muon
 
@@ -105,6 +111,16 @@ extern "C" muon_status muon_momentum_norm_noalloc(int rows, int cols, int grad_d
                  (unsigned long long)MUON_NOALLOC_MAX_BLOCKS * NA_ELEMS_PER_BLOCK);
         put_msg(err_msg, err_cap, msg);
         return MUON_ERR_UNSUPPORTED;
+    }
+    // B and U_out are written (and declared __restrict__ in the kernel): neither may
+    // share memory with another buffer of the call; the one-float norm neither
+    const size_t gbytes = total * (grad_dtype == MUON_BF16 ? 2 : 4), fbytes = total * 4;
+    if (spans_overlap(B, fbytes, G, gbytes) || (U_out && (spans_overlap(U_out, fbytes, G, gbytes) ||
+                                                          spans_overlap(U_out, fbytes, B, fbytes))) ||
+        spans_overlap(norm_out, 4, G, gbytes) || spans_overlap(norm_out, 4, B, fbytes) ||
+        (U_out && spans_overlap(norm_out, 4, U_out, fbytes))) {
+        put_msg(err_msg, err_cap, "B, U_out and norm_out are written: they may not overlap each other or G");
+        return MUON_ERR_INVALID;
     }
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NA_MAX_DEVICES) {

@@ -278,6 +278,7 @@ def test_qk_clip_binding_checks_tensors_before_the_library():
     import torch
     opt = mb.Muon.__new__(mb.Muon)               # no device handle: nothing may reach the library
     opt._h = ctypes.c_void_p()
+    opt.device = 0
     Wq = torch.zeros(8, 4)
     S = torch.ones(2)
     with pytest.raises(ValueError):
@@ -295,6 +296,7 @@ def test_binding_checks_buffer_dtypes_before_the_library():
     import torch
     opt = mb.Muon.__new__(mb.Muon)
     opt._h = ctypes.c_void_p()
+    opt.device = 0
     W, B = torch.zeros(4, 8), torch.zeros(4, 8)
     G = torch.zeros(4, 8, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
@@ -305,3 +307,51 @@ def test_binding_checks_buffer_dtypes_before_the_library():
         opt.step_host([mb.Group(W=[W, W.clone()], G=[G, G.float()], B=[B, B.clone()])])
     with pytest.raises(ValueError):
         opt.last_update(0, 0, torch.zeros(4, 8))              # no call has recorded any matrix
+
+
+class _FakeCudaTensor:
+    """Stands in for a CUDA tensor on a machine without a GPU: just the attributes
+    the binding inspects before it calls the library."""
+
+    def __init__(self, shape, dtype, index):
+        self.shape, self.dtype, self.is_cuda = tuple(shape), dtype, True
+        self.device = torch.device("cuda", index)
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):
+        raise AssertionError("a wrong-device tensor reached the library call")
+
+    def numel(self):
+        return int(np.prod(self.shape))
+
+
+def test_binding_refuses_tensors_of_another_device():
+    """The kernels of a handle run on its device and take only that device's memory:
+    a W, G, B, output or building-block buffer on another GPU is refused by the
+    binding before any call into the library.  The no-allocation call takes its
+    device from B and refuses the other buffers when they live elsewhere."""
+    opt = mb.Muon.__new__(mb.Muon)
+    opt._h = ctypes.c_void_p()
+    opt.device = 0
+    f32, bf = torch.float32, torch.bfloat16
+    on0 = lambda dt=f32: _FakeCudaTensor((4, 8), dt, 0)
+    on1 = lambda dt=f32: _FakeCudaTensor((4, 8), dt, 1)
+    for W, G, B in ((on1(), on0(bf), on0()), (on0(), on1(bf), on0()), (on0(), on0(bf), on1())):
+        with pytest.raises(ValueError, match="cuda:1"):
+            opt.step([mb.Group(W=[W], G=[G], B=[B])])
+    with pytest.raises(ValueError, match="cuda:1"):
+        opt.orthogonalize([([on0()], [on1()])])
+    with pytest.raises(ValueError, match="cuda:0"):
+        opt.ns_phase(mb.NS_GRAM, mb.PREC_BF16, 8, 8, 1, 1.0, 0.0, x_op=on1(bf), out=on0(bf))
+    opt._shapes = [(4, 8, 1)]
+    with pytest.raises(ValueError, match="cuda:1"):
+        opt.last_update(0, 0, on1())
+    n1 = _FakeCudaTensor((1,), f32, 1)
+    with pytest.raises(ValueError, match="cuda:1"):
+        mb.momentum_norm_noalloc(on1(bf), on0(), _FakeCudaTensor((1,), f32, 0))
+    with pytest.raises(ValueError, match="cuda:1"):
+        mb.momentum_norm_noalloc(on0(bf), on0(), n1)
+    with pytest.raises(ValueError, match="cuda:1"):
+        mb.momentum_norm_noalloc(on0(bf), on0(), _FakeCudaTensor((1,), f32, 0), U_out=on1())

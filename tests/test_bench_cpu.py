@@ -27,9 +27,35 @@ def test_cpu_baseline_record():
 
 
 def test_elementwise_bytes_per_element():
+    """The method's count for the momentum kernel: G 2 (bf16) or 4 (fp32), B 4 + 4,
+    X0 2 = 12 (14) B/elem; the bf16-pair iterate moves 2 B/elem more."""
     w = wl.get("square4096")
-    mom, app = bench.elementwise_bytes(w)
-    assert mom == 14 * w.elements          # G 2, B 4 + 4, X hi 2 + lo 2
+    mom, moved, app = bench.elementwise_bytes(w)
+    assert mom == 12 * w.elements and moved == 14 * w.elements and app == 12 * w.elements
+    t = wl.get("tiny")
+    assert bench.elementwise_bytes(t)[0] == 14 * t.elements
+
+
+def test_ns_figures_follow_their_stated_counts():
+    """Every fraction in the bench line can be recomputed from the line's own fields."""
+    w = wl.get("square4096")
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
+    steps = 4
+    phases = {"momentum_norm": (0.2, 4), "norm_finalize": (0.0, 0), "gram": (1.2, 20), "poly": (1.2, 20),
+              "update": (2.0, 20), "apply": (0.0, 0)}
+    f = bench.ns_figures(w, 1.25, 1.10, phases, steps, peaks)
+    m = 4096.0
+    sym = 5 * (3 * m ** 3 + m ** 3)
+    assert f["ns5_symmetric"]["flops_per_step"] == sym
+    assert abs(f["ns5_symmetric"]["ns_ms_per_step"] - (1.25 - 0.05)) < 1e-9
+    assert abs(f["ns5_symmetric"]["tflops"] - round(sym / 1.2e-3 / 1e12, 2)) < 1e-6
+    assert abs(f["ns5_symmetric"]["frac_sustained"] - round(sym / 1.2e-3 / 1e12 / 1400.0, 4)) < 1e-9
+    assert abs(f["ns5_symmetric"]["tflops_burst"] - round(sym / 1.05e-3 / 1e12, 2)) < 1e-6
+    assert abs(f["momentum_gbs"] - round(12 * w.elements / 0.05e-3 / 1e9, 1)) < 1e-6
+    assert f["momentum_bytes_per_elem"] == 12 and f["momentum_moved_bytes_per_elem"] == 14
+    nominal = 5 * (4 * m ** 3 + 2 * m ** 3)
+    assert abs(f["ns5_tflops_nominal"] - round(nominal / 1.25e-3 / 1e12, 2)) < 1e-6
+    assert abs(f["ns5_tflops_phase_sum"] - round(nominal / 1.1e-3 / 1e12, 2)) < 1e-6
 
 
 def _ranks_worker(rank, world, port, out_dir):

@@ -61,3 +61,34 @@ def test_noalloc_rejects_oversize_and_bad_arguments():
     st = L.muon_momentum_norm_noalloc(rows, cols, mb.MUON_FP32, G.data_ptr(), B.data_ptr(), None, 0.9, 1,
                                       n.data_ptr(), None, err, 256)
     assert st == mb.MUON_ERR_UNSUPPORTED and b"no-allocation limit" in err.value
+    # written buffers may not overlap: U_out is B, U_out inside G, norm inside B
+    for u, nrm in ((B, n), (G, n), (None, B[0, :1])):
+        with pytest.raises(mb.MuonError) as e:
+            mb.momentum_norm_noalloc(G, B, nrm, U_out=u)
+        assert e.value.status == mb.MUON_ERR_INVALID
+    st = L.muon_momentum_norm_noalloc(8, 8, mb.MUON_FP32, G.data_ptr(), G.data_ptr() + 16, None, 0.9, 1,
+                                      n.data_ptr(), None, err, 256)
+    assert st == mb.MUON_ERR_INVALID and b"overlap" in err.value
+
+
+def test_noalloc_calls_leave_free_device_memory_unchanged():
+    """After one warm-up call (which may load the module and place the static array),
+    further calls take no device memory: the free bytes the driver reports stay the
+    same across calls, and torch's allocator holds no more than before."""
+    mbuild.build()
+    torch.cuda.set_device(0)
+    rows, cols = 2048, 1536
+    G = torch.randn(rows, cols, device="cuda").to(torch.bfloat16)
+    B = torch.zeros(rows, cols, device="cuda")
+    U = torch.empty(rows, cols, device="cuda")
+    n = torch.empty(1, device="cuda")
+    mb.momentum_norm_noalloc(G, B, n, U_out=U)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    held0 = torch.cuda.memory_reserved()
+    for _ in range(5):
+        mb.momentum_norm_noalloc(G, B, n, U_out=U)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert free1 == free0
+    assert torch.cuda.memory_reserved() == held0

@@ -268,3 +268,57 @@ def parity_subset(wl: Workload) -> List[int]:
 def random_orthogonal(n: int, seed: int) -> np.ndarray:
     """Haar n x n orthogonal matrix (for invariance tests)."""
     return _haar_columns(np.random.default_rng(seed), n, n)
+
+
+# --------------------------------------------------------------------------- on-device draws (benchmark)
+
+def _torch_seed(w: int, step: int, k: int, stream: int) -> int:
+    base = 1234 + 1000 * w + (step if stream == 1 else 0)
+    return (base * 1_000_003 + k) * 4 + stream
+
+
+def device_tensors(wl: Workload, step: int, device, dtype_grad: bool = True):
+    """The workload's gradients at `step` and initial weights drawn on a CUDA device
+    with torch's generator: the same recipe as grad_fp32 / weight (shapes, value
+    distribution, spectrum, spike, heavy rows), a different random stream.  For the
+    benchmark's large workloads, whose numpy draws take tens of seconds; parity tests
+    use the numpy draws above.  Returns (weights fp32, gradients bf16 or fp32)."""
+    import torch
+    gen = torch.Generator(device=device)
+
+    def randn(shape, seed):
+        gen.manual_seed(seed)
+        return torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+
+    def haar(n, k, seed):
+        q, r = torch.linalg.qr(randn((n, k), seed))
+        return q * torch.sign(torch.diagonal(r))[None, :]
+
+    Ws, Gs = [], []
+    for k, spec in enumerate(wl.matrices):
+        r, c = spec.rows, spec.cols
+        Ws.append(0.02 * randn((r, c), _torch_seed(wl.index, 0, k, 2)))
+        s1 = _torch_seed(wl.index, step, k, 1)
+        if wl.grad_kind == "iid":
+            g = randn((r, c), s1)
+        elif wl.grad_kind in ("lowrank", "powerlaw"):
+            m = min(r, c)
+            expo = 1.5 if wl.grad_kind == "lowrank" else 1.0
+            sigma = torch.arange(1, m + 1, device=device, dtype=torch.float32) ** (-expo)
+            sigma *= math.sqrt(r * c) / torch.linalg.vector_norm(sigma)
+            g = (haar(r, m, s1) * sigma[None, :]) @ haar(c, m, s1 + 1).T
+            if wl.grad_kind == "lowrank":
+                g += 0.01 * randn((r, c), s1 + 2)
+        elif wl.grad_kind == "spike":
+            sigma_edge = (math.sqrt(r) + math.sqrt(c)) / math.sqrt(c)
+            g = randn((r, c), s1) * (1.0 / math.sqrt(c))
+            g += (10.0 * sigma_edge) * (haar(r, 8, s1 + 1) @ haar(c, 8, s1 + 2).T)
+        elif wl.grad_kind == "heavy_rows":
+            g = randn((r, c), s1)
+            gen.manual_seed(s1 + 1)
+            heavy = torch.randperm(r, generator=gen, device=device)[: int(math.ceil(0.01 * r))]
+            g[heavy, :] *= 20.0
+        else:
+            raise ValueError(wl.grad_kind)
+        Gs.append(g.to(torch.bfloat16) if (dtype_grad and wl.grad_dtype == BF16) else g)
+    return Ws, Gs
