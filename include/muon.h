@@ -139,6 +139,43 @@ muon_status muon_step(muon_handle* h, const muon_group* groups, int n_groups, vo
  * buffers must stay untouched until the stream reaches the end of the call. */
 muon_status muon_step_host(muon_handle* h, const muon_group* groups, int n_groups, void* stream);
 
+/* The step without its weight update, for callers that apply the update
+ * themselves (the data-parallel sharded step: each rank computes the update
+ * direction of the matrices it owns, the ranks exchange O, and every rank applies
+ * every O with muon_apply).  B <- mu*B + G and the Newton-Schulz direction O are
+ * computed exactly as in muon_step; O (rows x cols, de-oriented, scale s not
+ * applied) is written to O[k] in out_dtype -- fp32, or bf16 rounded to nearest --
+ * and W is neither read nor written.  G: bf16 or fp32, read only; B: fp32,
+ * updated in place; O: device buffers, written.  B and O may not overlap any
+ * buffer of the call (MUON_ERR_INVALID).  Same conventions as muon_group. */
+typedef struct {
+    int rows, cols, count;
+    int grad_dtype;          /* muon_dtype of G */
+    int out_dtype;           /* muon_dtype of O */
+    const void* const* G;
+    float* const* B;
+    void* const* O;
+} muon_direction_group;
+
+muon_status muon_step_direction(muon_handle* h, const muon_direction_group* groups, int n_groups, void* stream);
+
+/* The weight update of eq. 3 with result 2's decay and scale, from a caller's O:
+ * W <- W - lr*wd*W - lr*s*O for every matrix, with the handle's lr, weight_decay and
+ * scale mode (s from the shape for MATCH_RMS, group.scale for CUSTOM, 1 for NONE).
+ * W: fp32 rows x cols, device, updated in place; O: rows x cols in o_dtype (fp32 or
+ * bf16), device, read only.  No W may overlap any W or O of the call
+ * (MUON_ERR_INVALID).  The first call with a new set of pointers uploads a small
+ * table and synchronises the stream. */
+typedef struct {
+    int rows, cols, count;
+    int o_dtype;             /* muon_dtype of O */
+    float scale;             /* MUON_SCALE_CUSTOM only */
+    float* const* W;
+    const void* const* O;
+} muon_apply_group;
+
+muon_status muon_apply(muon_handle* h, const muon_apply_group* groups, int n_groups, void* stream);
+
 /* Orthogonalisation alone: O = NS_k(M / (||M||_F + eps)) per matrix, with the
  * orientation rule of section 4 and the handle's ns_steps / coefficients /
  * precision.  M: bf16 or fp32 rows x cols (device, read only); O: fp32 rows x cols

@@ -46,6 +46,19 @@ class _OrthoGroup(ctypes.Structure):
                 ("O", ctypes.POINTER(ctypes.c_void_p))]
 
 
+class _DirGroup(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("cols", ctypes.c_int), ("count", ctypes.c_int),
+                ("grad_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+                ("G", ctypes.POINTER(ctypes.c_void_p)), ("B", ctypes.POINTER(ctypes.c_void_p)),
+                ("O", ctypes.POINTER(ctypes.c_void_p))]
+
+
+class _ApplyGroup(ctypes.Structure):
+    _fields_ = [("rows", ctypes.c_int), ("cols", ctypes.c_int), ("count", ctypes.c_int),
+                ("o_dtype", ctypes.c_int), ("scale", ctypes.c_float),
+                ("W", ctypes.POINTER(ctypes.c_void_p)), ("O", ctypes.POINTER(ctypes.c_void_p))]
+
+
 class _PhaseArgs(ctypes.Structure):
     _fields_ = [("phase", ctypes.c_int), ("precision", ctypes.c_int), ("m", ctypes.c_int), ("n", ctypes.c_int),
                 ("count", ctypes.c_int), ("alpha", ctypes.c_float), ("beta", ctypes.c_float),
@@ -66,6 +79,8 @@ _SIGNATURES = {
     "muon_memory_held": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(ctypes.c_size_t)]),
     "muon_step": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_Group), ctypes.c_int, ctypes.c_void_p]),
     "muon_step_host": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_Group), ctypes.c_int, ctypes.c_void_p]),
+    "muon_step_direction": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_DirGroup), ctypes.c_int, ctypes.c_void_p]),
+    "muon_apply": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_ApplyGroup), ctypes.c_int, ctypes.c_void_p]),
     "muon_orthogonalize": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_OrthoGroup), ctypes.c_int, ctypes.c_void_p]),
     "muon_ns_phase_run": (ctypes.c_int, [ctypes.c_void_p, ctypes.POINTER(_PhaseArgs), ctypes.c_void_p]),
     "muon_qk_clip": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
@@ -238,6 +253,51 @@ class Muon:
         arr, keep = self._groups(groups, False)
         self._shapes = [(arr[i].rows, arr[i].cols, arr[i].count) for i in range(len(groups))]
         self._check(lib().muon_step_host(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream, self.device))), "muon_step_host")
+
+    def step_direction(self, groups, stream=None):
+        """groups: list of (G_list, B_list, O_list) of same-shape matrices.  B is updated
+        and O (fp32 or bf16 tensors of W's shape) receives the Newton-Schulz direction;
+        no weight is touched (see muon_step_direction)."""
+        import torch
+        arr = (_DirGroup * len(groups))()
+        keep = []
+        for i, (Gs, Bs, Os) in enumerate(groups):
+            rows, cols = Bs[0].shape
+            if not (len(Gs) == len(Bs) == len(Os)):
+                raise ValueError("G, B and O lists differ in length")
+            _check_tensors(Gs, (rows, cols), True, Gs[0].dtype, self.device)
+            _check_tensors(Bs, (rows, cols), True, torch.float32, self.device)
+            _check_tensors(Os, (rows, cols), True, Os[0].dtype, self.device)
+            pg, pb, po = _ptrs(Gs), _ptrs(Bs), _ptrs(Os)
+            keep += [pg, pb, po]
+            arr[i] = _DirGroup(rows, cols, len(Bs), _dtype_code(Gs[0]), _dtype_code(Os[0]),
+                               ctypes.cast(pg, ctypes.POINTER(ctypes.c_void_p)),
+                               ctypes.cast(pb, ctypes.POINTER(ctypes.c_void_p)),
+                               ctypes.cast(po, ctypes.POINTER(ctypes.c_void_p)))
+        self._check(lib().muon_step_direction(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream, self.device))),
+                    "muon_step_direction")
+
+    def apply(self, groups, stream=None):
+        """groups: list of (W_list, O_list[, scale]) of same-shape matrices:
+        W <- W - lr*wd*W - lr*s*O (see muon_apply); O fp32 or bf16."""
+        import torch
+        arr = (_ApplyGroup * len(groups))()
+        keep = []
+        for i, grp in enumerate(groups):
+            Ws, Os = grp[0], grp[1]
+            scale = float(grp[2]) if len(grp) > 2 else 1.0
+            rows, cols = Ws[0].shape
+            if len(Ws) != len(Os):
+                raise ValueError("W and O lists differ in length")
+            _check_tensors(Ws, (rows, cols), True, torch.float32, self.device)
+            _check_tensors(Os, (rows, cols), True, Os[0].dtype, self.device)
+            pw, po = _ptrs(Ws), _ptrs(Os)
+            keep += [pw, po]
+            arr[i] = _ApplyGroup(rows, cols, len(Ws), _dtype_code(Os[0]), scale,
+                                 ctypes.cast(pw, ctypes.POINTER(ctypes.c_void_p)),
+                                 ctypes.cast(po, ctypes.POINTER(ctypes.c_void_p)))
+        self._check(lib().muon_apply(self._h, arr, len(groups), ctypes.c_void_p(_stream(stream, self.device))),
+                    "muon_apply")
 
     def orthogonalize(self, groups, stream=None):
         """groups: list of (M_list, O_list); O = NS(M / (||M||_F + eps)), fp32 outputs."""

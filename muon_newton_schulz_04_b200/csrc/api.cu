@@ -116,6 +116,9 @@ struct muon_handle {
     unsigned long long g_version = 0;
     unsigned long long plans_built = 0;
     cudaEvent_t ev_start = nullptr, ev_w = nullptr, ev_k1 = nullptr, ev_done = nullptr;
+    // muon_apply: segment table of the last call (device copy in apply_segs)
+    DevBuf apply_segs;
+    std::vector<EwSeg> apply_uploaded;
 };
 
 namespace {
@@ -290,7 +293,7 @@ muon_status ensure_buf(muon_handle* h, DevBuf& b, size_t bytes) {
         b.ptr = nullptr;
         b.size = 0;
     }
-    const size_t held = h->ws.size + h->staging.size + h->scratch.size;   // b is already released
+    const size_t held = h->ws.size + h->staging.size + h->scratch.size + h->apply_segs.size;   // b is already released
     if (h->mem_limit != 0 && held + bytes > h->mem_limit)
         return fail(h, MUON_ERR_OOM, "device buffers of %zu bytes would exceed the handle's memory limit of %zu bytes",
                     held + bytes, h->mem_limit);
@@ -338,12 +341,11 @@ muon_status encode_map(muon_handle* h, CUtensorMap* m, const void* base, int col
     return encode_map_box(h, m, base, cols, rows, count, ld, 64, box_rows, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-// 32-row boxes of the UPDATE epilogue (tc_gemm_epi_cols() columns, the swizzle whose
-// span is one box row).
+// Boxes of the UPDATE epilogue: tc_gemm_epi_rows() x tc_gemm_epi_cols() (32 bf16
+// columns, one 64-byte row), with the 64-byte swizzle whose span is one box row.
 muon_status encode_epi_map(muon_handle* h, CUtensorMap* m, const void* base, int cols, int rows, int count, int ld) {
-    const int bc = tc_gemm_epi_cols();
-    return encode_map_box(h, m, base, cols, rows, count, ld, bc, 32,
-                          bc == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+    return encode_map_box(h, m, base, cols, rows, count, ld, tc_gemm_epi_cols(), tc_gemm_epi_rows(),
+                          CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 bool is_bf16_path(const muon_handle* h) { return h->cfg.precision == MUON_PREC_BF16; }
@@ -565,7 +567,7 @@ float update_scale(const muon_handle* h, int rows, int cols, float custom) {
 }
 
 // Fills the caller-pointer part of the segment table and uploads it if it changed.
-struct MatPtrs { const void* g; float* b; float* w; int g_bf16; float scale; };
+struct MatPtrs { const void* g; float* b; float* w; int g_bf16; float scale; int out_bf16 = 0; };
 
 muon_status upload_segs(muon_handle* h, const std::vector<MatPtrs>& mp, cudaStream_t s) {
     Plan& P = h->plan;
@@ -582,6 +584,7 @@ muon_status upload_segs(muon_handle* h, const std::vector<MatPtrs>& mp, cudaStre
             sg.g = mp[mi].g; sg.b = mp[mi].b; sg.w = mp[mi].w;
             sg.g_bf16 = mp[mi].g_bf16;
             sg.update_scale = mp[mi].scale;
+            sg.out_bf16 = mp[mi].out_bf16;
             if (bf16) {
                 sg.o_hi = reinterpret_cast<const __nv_bfloat16*>(base + P.offs[g].xb[h->cfg.ns_steps & 1]) + (size_t)z * xe;
                 sg.o_lo = reinterpret_cast<const __nv_bfloat16*>(base + P.offs[g].xl) + (size_t)z * xe;
@@ -694,7 +697,7 @@ muon_status run_graph_or_direct(muon_handle* h, bool momentum, bool copy_out, cu
     const bool use_graph = h->graphs && !h->timing && !hooks && cs == cudaStreamCaptureStatusNone &&
                            !(h->pair && tc_gemm_split_tiles());
     if (!use_graph) return run_pipeline(h, momentum, copy_out, s, hooks);
-    const int mode = copy_out ? 1 : 0;
+    const int mode = (copy_out ? 1 : 0) | (momentum ? 2 : 0);
     const bool same = h->gexec && h->g_mode == mode && h->g_ws == h->ws.ptr && h->g_version == P.version &&
                       std::memcmp(&h->g_cfg, &h->cfg, sizeof(muon_config)) == 0 && h->g_segs.size() == P.uploaded.size() &&
                       std::memcmp(h->g_segs.data(), P.uploaded.data(), P.uploaded.size() * sizeof(EwSeg)) == 0;
@@ -817,7 +820,7 @@ muon_status muon_set_memory_limit(muon_handle* h, size_t bytes) {
 
 muon_status muon_memory_held(const muon_handle* h, size_t* bytes) {
     if (!h || !bytes) return MUON_ERR_INVALID;
-    *bytes = h->ws.size + h->staging.size + h->scratch.size;
+    *bytes = h->ws.size + h->staging.size + h->scratch.size + h->apply_segs.size;
     return MUON_OK;
 }
 
@@ -906,6 +909,113 @@ muon_status muon_step_host(muon_handle* h, const muon_group* groups, int n_group
     }
     CUDA_TRY(h, cudaEventRecord(h->ev_done, h->side));
     CUDA_TRY(h, cudaStreamWaitEvent(s, h->ev_done, 0));
+    return MUON_OK;
+}
+
+muon_status muon_step_direction(muon_handle* h, const muon_direction_group* groups, int n_groups, void* stream) {
+    if (!h) return MUON_ERR_INVALID;
+    NvtxRange nr("muon_step_direction");
+    if (!groups || n_groups <= 0) return fail(h, MUON_ERR_INVALID, "groups must be a non-empty array");
+    std::vector<int> shapes;
+    std::vector<MatPtrs> mp;
+    std::vector<Span> sp;
+    long long total = 0;
+    for (int i = 0; i < n_groups; ++i) {
+        const muon_direction_group& g = groups[i];
+        std::string why;
+        if (check_shape(g.rows, g.cols, g.count, &why) != MUON_OK) return fail(h, MUON_ERR_INVALID, "group %d: %s", i, why.c_str());
+        if (g.grad_dtype != MUON_BF16 && g.grad_dtype != MUON_FP32) return fail(h, MUON_ERR_INVALID, "group %d: bad grad_dtype", i);
+        if (g.out_dtype != MUON_BF16 && g.out_dtype != MUON_FP32) return fail(h, MUON_ERR_INVALID, "group %d: bad out_dtype", i);
+        if (!g.G || !g.B || !g.O) return fail(h, MUON_ERR_INVALID, "group %d: G, B and O arrays are required", i);
+        total += g.count;
+        if (total > (1 << 24)) return fail(h, MUON_ERR_INVALID, "too many matrices");
+        shapes.push_back(g.rows); shapes.push_back(g.cols); shapes.push_back(g.count);
+        const uintptr_t e = (uintptr_t)g.rows * (uintptr_t)g.cols;
+        const size_t gsz = g.grad_dtype == MUON_BF16 ? 2 : 4, osz = g.out_dtype == MUON_BF16 ? 2 : 4;
+        for (int k = 0; k < g.count; ++k) {
+            if (!g.G[k] || !g.B[k] || !g.O[k]) return fail(h, MUON_ERR_INVALID, "group %d: NULL pointer at %d", i, k);
+            if (!aligned(g.B[k], 4) || !aligned(g.G[k], gsz) || !aligned(g.O[k], osz))
+                return fail(h, MUON_ERR_INVALID, "group %d: misaligned pointer at %d", i, k);
+            const uintptr_t b = (uintptr_t)g.B[k], gg = (uintptr_t)g.G[k], o = (uintptr_t)g.O[k];
+            sp.push_back(Span{b, b + 4 * e, true, i, k, 'B'});
+            sp.push_back(Span{o, o + osz * e, true, i, k, 'O'});
+            sp.push_back(Span{gg, gg + gsz * e, false, i, k, 'G'});
+            MatPtrs m{g.G[k], g.B[k], reinterpret_cast<float*>(g.O[k]), g.grad_dtype == MUON_BF16 ? 1 : 0, 1.0f,
+                      g.out_dtype == MUON_BF16 ? 1 : 0};
+            mp.push_back(m);
+        }
+    }
+    {
+        std::string why;
+        if (check_spans(sp, &why) != MUON_OK) return fail(h, MUON_ERR_INVALID, "%s", why.c_str());
+    }
+    DeviceGuard dg(h->device);
+    h->last_error.clear();
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    muon_status st = ensure_plan(h, shapes, s);
+    if (st != MUON_OK) return st;
+    if ((st = upload_segs(h, mp, s)) != MUON_OK) return st;
+    return run_graph_or_direct(h, true, true, s, nullptr);
+}
+
+muon_status muon_apply(muon_handle* h, const muon_apply_group* groups, int n_groups, void* stream) {
+    if (!h) return MUON_ERR_INVALID;
+    NvtxRange nr("muon_apply");
+    if (!groups || n_groups <= 0) return fail(h, MUON_ERR_INVALID, "groups must be a non-empty array");
+    std::vector<EwSeg> segs;
+    std::vector<Span> sp;
+    int blocks = 0;
+    for (int i = 0; i < n_groups; ++i) {
+        const muon_apply_group& g = groups[i];
+        std::string why;
+        if (check_shape(g.rows, g.cols, g.count, &why) != MUON_OK) return fail(h, MUON_ERR_INVALID, "group %d: %s", i, why.c_str());
+        if (g.o_dtype != MUON_BF16 && g.o_dtype != MUON_FP32) return fail(h, MUON_ERR_INVALID, "group %d: bad o_dtype", i);
+        if (!finite(g.scale)) return fail(h, MUON_ERR_INVALID, "group %d: scale is not finite", i);
+        if (!g.W || !g.O) return fail(h, MUON_ERR_INVALID, "group %d: W and O arrays are required", i);
+        const uintptr_t e = (uintptr_t)g.rows * (uintptr_t)g.cols;
+        const size_t osz = g.o_dtype == MUON_BF16 ? 2 : 4;
+        const float sc = update_scale(h, g.rows, g.cols, g.scale);
+        const int nb = (int)((e + EW_FLAT_ELEMS - 1) / EW_FLAT_ELEMS);
+        for (int k = 0; k < g.count; ++k) {
+            if (!g.W[k] || !g.O[k]) return fail(h, MUON_ERR_INVALID, "group %d: NULL pointer at %d", i, k);
+            if (!aligned(g.W[k], 4) || !aligned(g.O[k], osz)) return fail(h, MUON_ERR_INVALID, "group %d: misaligned pointer at %d", i, k);
+            if ((long long)blocks + nb > (1ll << 31) - 1) return fail(h, MUON_ERR_INVALID, "too many elements");
+            const uintptr_t w = (uintptr_t)g.W[k], o = (uintptr_t)g.O[k];
+            sp.push_back(Span{w, w + 4 * e, true, i, k, 'W'});
+            sp.push_back(Span{o, o + osz * e, false, i, k, 'O'});
+            EwSeg sg{};
+            sg.w = g.W[k];
+            if (g.o_dtype == MUON_BF16) sg.o_hi = static_cast<const __nv_bfloat16*>(g.O[k]);
+            else sg.o_src = static_cast<const float*>(g.O[k]);
+            sg.rows = g.rows; sg.cols = g.cols; sg.ldn = g.cols; sg.transposed = 0;
+            sg.vec = (g.cols % 8 == 0) && aligned(g.W[k], 16) && aligned(g.O[k], 16) ? 1 : 0;
+            sg.apply_begin = blocks; sg.apply_count = nb; blocks += nb;
+            sg.mat = (int)segs.size();
+            sg.update_scale = sc;
+            segs.push_back(sg);
+        }
+    }
+    {
+        std::string why;
+        if (check_spans(sp, &why) != MUON_OK) return fail(h, MUON_ERR_INVALID, "%s", why.c_str());
+    }
+    DeviceGuard dg(h->device);
+    h->last_error.clear();
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool same = h->apply_uploaded.size() == segs.size() &&
+                      std::memcmp(h->apply_uploaded.data(), segs.data(), segs.size() * sizeof(EwSeg)) == 0;
+    if (!same) {
+        // the table may still be read by an earlier launch on another stream
+        if (h->apply_segs.ptr) CUDA_TRY(h, cudaDeviceSynchronize());
+        muon_status st = ensure_buf(h, h->apply_segs, segs.size() * sizeof(EwSeg));
+        if (st != MUON_OK) return st;
+        CUDA_TRY(h, cudaMemcpyAsync(h->apply_segs.ptr, segs.data(), segs.size() * sizeof(EwSeg), cudaMemcpyHostToDevice, s));
+        CUDA_TRY(h, cudaStreamSynchronize(s));
+        h->apply_uploaded = segs;
+    }
+    const muon_config& c = h->cfg;
+    TIMED(h, 5, s, launch_apply(static_cast<const EwSeg*>(h->apply_segs.ptr), (int)segs.size(), blocks,
+                                1.f - c.lr * c.weight_decay, c.lr, nullptr, 0, s));
     return MUON_OK;
 }
 
@@ -1199,6 +1309,7 @@ muon_status muon_destroy(muon_handle* h) {
         if (h->ws.ptr) cudaFree(h->ws.ptr);
         if (h->staging.ptr) cudaFree(h->staging.ptr);
         if (h->scratch.ptr) cudaFree(h->scratch.ptr);
+        if (h->apply_segs.ptr) cudaFree(h->apply_segs.ptr);
         if (h->d_err) cudaFree(h->d_err);
     }
     delete h;

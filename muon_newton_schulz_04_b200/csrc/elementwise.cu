@@ -75,6 +75,11 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
     lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
+__device__ __forceinline__ uint32_t pack2_bf16(float a, float b) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
 __device__ __forceinline__ void store_x0(const EwSeg& sg, size_t xo, float u, int bf16_operand) {
     if (bf16_operand) {
         const __nv_bfloat16 h = __float2bfloat16_rn(u);
@@ -85,9 +90,18 @@ __device__ __forceinline__ void store_x0(const EwSeg& sg, size_t xo, float u, in
     }
 }
 
-// Element i (index into the oriented m x ldn iterate) of the final X.
+// Element i (index into the oriented m x ldn iterate) of the final X: the bf16 pair
+// o_hi + o_lo, o_hi alone (a bf16 O given to muon_apply), or fp32 o_src.
 __device__ __forceinline__ float load_o(const EwSeg& sg, size_t i) {
-    return sg.o_hi ? __bfloat162float(sg.o_hi[i]) + __bfloat162float(sg.o_lo[i]) : sg.o_src[i];
+    if (sg.o_hi) return __bfloat162float(sg.o_hi[i]) + (sg.o_lo ? __bfloat162float(sg.o_lo[i]) : 0.f);
+    return sg.o_src[i];
+}
+
+// Copy-out of one value of O to element i of the destination (fp32, or bf16 when
+// the segment asks for it).
+__device__ __forceinline__ void store_out(const EwSeg& sg, float* dst, size_t i, float v) {
+    if (sg.out_bf16) reinterpret_cast<__nv_bfloat16*>(dst)[i] = __float2bfloat16_rn(v);
+    else dst[i] = v;
 }
 
 __global__ void __launch_bounds__(EW_THREADS, EW_MIN_BLOCKS) momentum_norm_kernel(const EwSeg* __restrict__ segs, int nseg,
@@ -330,7 +344,7 @@ __device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay
                 float4 o0, o1;
                 if (sg.o_hi) {
                     const uint4 h = *reinterpret_cast<const uint4*>(sg.o_hi + e);
-                    const uint4 l = *reinterpret_cast<const uint4*>(sg.o_lo + e);
+                    const uint4 l = sg.o_lo ? *reinterpret_cast<const uint4*>(sg.o_lo + e) : make_uint4(0u, 0u, 0u, 0u);
                     auto f = [](uint32_t a, uint32_t b, bool hi_half) {
                         return hi_half ? __uint_as_float(a & 0xFFFF0000u) + __uint_as_float(b & 0xFFFF0000u)
                                        : __uint_as_float(a << 16) + __uint_as_float(b << 16);
@@ -345,7 +359,13 @@ __device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay
                 float4* wp = reinterpret_cast<float4*>(dst + e);
                 if (copy_out) {
                     o0.x *= os; o0.y *= os; o0.z *= os; o0.w *= os; o1.x *= os; o1.y *= os; o1.z *= os; o1.w *= os;
-                    wp[0] = o0; wp[1] = o1;
+                    if (sg.out_bf16) {
+                        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dst) + e) =
+                            make_uint4(pack2_bf16(o0.x, o0.y), pack2_bf16(o0.z, o0.w), pack2_bf16(o1.x, o1.y),
+                                       pack2_bf16(o1.z, o1.w));
+                    } else {
+                        wp[0] = o0; wp[1] = o1;
+                    }
                 } else {
                     float4 w0 = wp[0], w1 = wp[1];
                     w0.x = fmaf(-step, o0.x * os, decay * w0.x); w0.y = fmaf(-step, o0.y * os, decay * w0.y);
@@ -359,7 +379,8 @@ __device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay
             for (size_t e = e0 + threadIdx.x; e < e1; e += EW_THREADS) {
                 const size_t r = e / (size_t)sg.cols, c = e - r * (size_t)sg.cols;
                 const float o = load_o(sg, r * (size_t)sg.ldn + c) * os;
-                dst[e] = copy_out ? o : fmaf(-step, o, decay * dst[e]);
+                if (copy_out) store_out(sg, dst, e, o);
+                else dst[e] = fmaf(-step, o, decay * dst[e]);
             }
         }
     } else {
@@ -379,7 +400,8 @@ __device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay
             if (i < sg.rows && j < sg.cols) {
                 const size_t e = (size_t)i * sg.cols + j;
                 const float o = tile[tx][ii] * os;
-                dst[e] = copy_out ? o : fmaf(-step, o, decay * dst[e]);
+                if (copy_out) store_out(sg, dst, e, o);
+                else dst[e] = fmaf(-step, o, decay * dst[e]);
             }
         }
     }
@@ -468,7 +490,10 @@ cudaError_t launch_apply(const EwSeg* segs, int nseg, int nblocks, float decay, 
 
 cudaError_t launch_copy_out_one(const EwSeg& seg, float* dst, const float* o_scale, cudaStream_t s) {
     if (seg.apply_count <= 0) return cudaSuccess;
-    return launch_pdl(copy_out_one_kernel, dim3(seg.apply_count), dim3(EW_THREADS), 0, s, seg, dst, o_scale);
+    EwSeg sg = seg;
+    sg.out_bf16 = 0;                  // the destination of this copy is fp32
+    if (reinterpret_cast<uintptr_t>(dst) % 16 != 0) sg.vec = 0;
+    return launch_pdl(copy_out_one_kernel, dim3(sg.apply_count), dim3(EW_THREADS), 0, s, sg, dst, o_scale);
 }
 
 }  // namespace muon

@@ -64,35 +64,38 @@ constexpr int S2_BM = 256, S2_BN = 256, S2_STAGES = MUON_S2_STAGES;
 constexpr int S2_A = 128 * BK * 2;            // 16 KiB: this CTA's 128 rows of A
 constexpr int S2_B = 128 * BK * 2;            // 16 KiB: this CTA's 128 columns of B
 
-// UPDATE epilogue of the two-CTA kernel: each epilogue warp streams its 32 rows of
-// the iterate through a private ring of EU_DEPTH shared-memory buffers, one
-// 32-row x EU_COLS-column box of hi and one of lo per buffer, loaded by TMA up to
-// EU_DEPTH - 1 chunks ahead (across tile boundaries) and written back in place, then
-// stored by TMA.  The operand ring of this mode is S2U_STAGES deep.
-#ifndef MUON_EU_COLS
-#define MUON_EU_COLS 32
-#endif
+// UPDATE epilogue of the two-CTA kernel: each column half of the CTA's 128 x 256
+// accumulator streams the iterate through a ring of EU_DEPTH shared-memory buffers,
+// each one 128-row x 32-column box of hi and one of lo (64-byte swizzle).  A TMA warp
+// per half (warps 10 and 11) loads the boxes up to EU_DEPTH - 1 chunks ahead, across
+// tile boundaries; the half's four compute warps rewrite each chunk in place, and
+// the TMA warp stores it once all four have arrived on the chunk's barrier.  The
+// operand ring of this mode is S2U_STAGES deep.
 #ifndef MUON_EU_DEPTH
 #define MUON_EU_DEPTH 3
 #endif
 #ifndef MUON_S2U_STAGES
 #define MUON_S2U_STAGES 4
 #endif
-constexpr int EU_COLS = MUON_EU_COLS;               // 16 or 32 columns per chunk
+constexpr int EU_COLS = 32;                         // columns per chunk: one 64-byte bf16 box row
+constexpr int EU_ROWS = 128;                        // rows per chunk: the CTA's accumulator rows
 constexpr int EU_DEPTH = MUON_EU_DEPTH;
-constexpr int EU_ROW_BYTES = EU_COLS * 2;           // one bf16 row of a box: 32 or 64 bytes
-constexpr int EU_BOX = 32 * EU_ROW_BYTES;           // one 32-row box
+constexpr int EU_ROW_BYTES = EU_COLS * 2;
+constexpr int EU_BOX = EU_ROWS * EU_ROW_BYTES;      // 8 KiB
 constexpr int EU_BUF = 2 * EU_BOX;                  // hi + lo
 constexpr int S2U_STAGES = MUON_S2U_STAGES;
-static_assert(EU_COLS == 16 || EU_COLS == 32, "epilogue chunks are 16 or 32 columns");
-static_assert(EU_DEPTH >= 2 && EU_DEPTH <= 8, "epilogue ring depth out of range");
+constexpr int NUM_THREADS_U = NUM_THREADS + 64;     // + the two epilogue TMA warps
+static_assert(EU_DEPTH >= 2 && EU_DEPTH <= 6, "epilogue ring depth out of range");
 
 constexpr int s2_stages(int mode) { return mode == MODE_UPDATE ? S2U_STAGES : S2_STAGES; }
-constexpr int s2_epi_bytes(int mode) { return mode == MODE_UPDATE ? NUM_EPI_WARPS * EU_DEPTH * EU_BUF : STAGE_BYTES; }
+constexpr int s2_epi_bytes(int mode) { return mode == MODE_UPDATE ? 2 * EU_DEPTH * EU_BUF : STAGE_BYTES; }
+constexpr int s2_threads(int mode) { return mode == MODE_UPDATE ? NUM_THREADS_U : NUM_THREADS; }
 // barriers: full / empty per stage, two tfull / tempty, drain, the epilogue ring's
 // (UPDATE), then the TMEM address and the abort flag
 constexpr int s2_bar_bytes(int mode) {
-    return (8 * (2 * s2_stages(mode) + 5 + (mode == MODE_UPDATE ? NUM_EPI_WARPS * EU_DEPTH : 0)) + 8 + 127) / 128 * 128;
+    // (+ UPDATE: the epilogue TMA warps' chunk coordinates, 2 x EU_DEPTH int4)
+    return (8 * (2 * s2_stages(mode) + 5 + (mode == MODE_UPDATE ? 4 * EU_DEPTH : 0)) + 8 + 16 +
+            (mode == MODE_UPDATE ? 2 * EU_DEPTH * 16 : 0) + 127) / 128 * 128;
 }
 // [operand ring][epilogue buffers][barriers]; the ring and the buffers are 1024-byte aligned
 constexpr int s2_smem(int mode) {
@@ -153,6 +156,15 @@ __device__ __forceinline__ void apply_chunk(const GemmParams& p, const GemmGroup
     float* w = sg.w;
     const float step = p.lr * sg.update_scale;
     const bool copy = p.apply_mode == 2;
+    if (copy && sg.out_bf16) {
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(sg.w);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int c = col0 + j;
+            if (c < gi.n) o[sg.transposed ? (size_t)c * sg.cols + row : (size_t)row * sg.cols + c] = __float2bfloat16_rn(val[j]);
+        }
+        return;
+    }
     if (!sg.transposed) {
         float* wr = w + (size_t)row * sg.cols;
         if (sg.vec && col0 + 31 < gi.n) {
@@ -226,6 +238,13 @@ __device__ __forceinline__ void apply_run8(const GemmParams& p, const EwSeg& sg,
     float* wr = sg.w + (size_t)r * sg.cols + c;
     const float step = p.lr * sg.update_scale;
     const bool copy = p.apply_mode == 2;
+    if (copy && sg.out_bf16) {
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(sg.w) + (size_t)r * sg.cols + c;
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            if (c + k < n) o[k] = __float2bfloat16_rn(val[k]);
+        return;
+    }
     if (sg.vec && c + 7 < n) {
         float4* w4 = reinterpret_cast<float4*>(wr);
 #pragma unroll
@@ -521,32 +540,41 @@ __device__ __forceinline__ void spin_ns(uint64_t ns) {
     while (globaltimer_ns() - t0 < ns) { }
 }
 
-// 32 lanes x 16 columns of 32-bit accumulators (lane i: row base_lane + i).
-__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32"
-        " {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr));
-}
-
-template <int NC>
-__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, uint32_t (&r)[NC]) {
-    if constexpr (NC == 32) tmem_ld_32x32b_x32(taddr, r);
-    else tmem_ld_32x32b_x16(taddr, r);
-}
-
 // Weight update (apply_mode 1) or copy-out (apply_mode 2) of NC finished values
 // O[row][col0 .. col0 + NC) of the oriented result, one row per lane.  A matrix that
 // was transposed for the smaller Gram gets W[c][row]: lanes hold consecutive rows,
 // so each store instruction of the warp covers 32 consecutive elements of W's row c.
 template <int NC>
 __device__ __forceinline__ void apply_row(const GemmParams& p, const GemmGroupInfo& gi, const EwSeg& sg, int row,
-                                          int col0, const float (&val)[NC]) {
+                                          int col0, const uint32_t (&bits)[NC]) {
+    float val[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) val[j] = __uint_as_float(bits[j]);
     float* w = sg.w;
     const float step = p.lr * sg.update_scale;
     const bool copy = p.apply_mode == 2;
+    if (copy && sg.out_bf16) {
+        __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(sg.w);
+        if (!sg.transposed) {
+            __nv_bfloat16* orow = o + (size_t)row * sg.cols;
+            if (sg.vec && col0 + NC - 1 < gi.n) {
+#pragma unroll
+                for (int qq = 0; qq < NC / 8; ++qq)
+                    *reinterpret_cast<uint4*>(orow + col0 + 8 * qq) =
+                        make_uint4(pack_bf16x2(val[8 * qq], val[8 * qq + 1]), pack_bf16x2(val[8 * qq + 2], val[8 * qq + 3]),
+                                   pack_bf16x2(val[8 * qq + 4], val[8 * qq + 5]), pack_bf16x2(val[8 * qq + 6], val[8 * qq + 7]));
+            } else {
+#pragma unroll
+                for (int j = 0; j < NC; ++j)
+                    if (col0 + j < gi.n) orow[col0 + j] = __float2bfloat16_rn(val[j]);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < NC; ++j)
+                if (col0 + j < gi.n) o[(size_t)(col0 + j) * sg.cols + row] = __float2bfloat16_rn(val[j]);
+        }
+        return;
+    }
     if (!sg.transposed) {
         float* wr = w + (size_t)row * sg.cols;
         if (sg.vec && col0 + NC - 1 < gi.n) {
@@ -582,10 +610,10 @@ __device__ __forceinline__ void apply_row(const GemmParams& p, const GemmGroupIn
     }
 }
 
-// Where chunk c of unit u lies for one epilogue warp of the two-CTA UPDATE kernel:
-// the warp's 32 rows (CTA `rank`, TMEM lane quarter q) and EU_COLS columns of its
-// column half.  A chunk is a "load chunk" when it needs the iterate (its unit is not
-// a split part that only stores a partial sum) and touches the matrix.
+// Where chunk c of a unit lies for one column half of the two-CTA UPDATE epilogue:
+// the CTA's 128 accumulator rows and EU_COLS columns of the half.  A chunk is a
+// "load chunk" when it needs the iterate (its unit is not a split part that only
+// stores a partial sum) and touches the matrix (gm x gn, the group's oriented shape).
 struct EuChunk {
     int g, mat, row0, col0, tcol;   // group, matrix, first row / column, TMEM column
     bool load;
@@ -595,27 +623,60 @@ __device__ __forceinline__ int eu_nchunks(int4 sk) {
     return (sk.z & 0xFF) == 2 ? 0 : ((sk.z >> 8) ? 64 : 128) / EU_COLS;
 }
 
-__device__ __forceinline__ EuChunk eu_chunk(const GemmParams& p, int4 tile, int4 sk, int c, int rank, int q,
-                                            int half) {
+__device__ __forceinline__ EuChunk eu_chunk(int4 tile, int4 sk, int gm, int gn, int c, int rank, int half) {
     const int nh = sk.z >> 8;
     EuChunk ch;
     ch.g = tile.x;
     ch.mat = tile.y;
-    ch.row0 = tile.z * S2_BM + rank * 128 + q * 32;
+    ch.row0 = tile.z * S2_BM + rank * 128;
     ch.tcol = half * (nh ? 64 : 128) + c * EU_COLS;
     ch.col0 = tile.w * S2_BN + (nh ? (nh - 1) * 128 : 0) + ch.tcol;
-    const GemmGroupInfo& gi = p.groups[tile.x];
-    ch.load = (sk.z & 0xFF) != 2 && ch.row0 < gi.m && ch.col0 < gi.n;
+    ch.load = (sk.z & 0xFF) != 2 && ch.row0 < gm && ch.col0 < gn;
     return ch;
 }
 
-// Byte offset of 16-byte slot k of row r inside a TMA box with EU_ROW_BYTES-byte rows
-// and the matching swizzle (64B: slot ^= (r >> 1) & 3; 32B: slot ^= (r >> 2) & 1).
+// Byte offset of 16-byte slot k of row r inside a box with 64-byte rows and the
+// 64-byte swizzle (slot ^= (r >> 1) & 3): the 8 lanes of a quarter-warp access read
+// 8 distinct slots of a 128-byte span, so the row-per-lane accesses are conflict free.
 __device__ __forceinline__ uint32_t eu_off(int r, int k) {
-    constexpr int NS = EU_ROW_BYTES / 16;
-    constexpr int SH = EU_ROW_BYTES == 64 ? 1 : 2;
-    return (uint32_t)(r * EU_ROW_BYTES + ((k ^ ((r >> SH) & (NS - 1))) << 4));
+    return (uint32_t)(r * EU_ROW_BYTES + ((k ^ ((r >> 1) & 3)) << 4));
 }
+
+// X' = alpha * acc + beta * (hi + lo) for this lane's row of one chunk, in place in
+// the swizzled hi / lo boxes at hi_s / lo_s; with APPLY, v[] is overwritten with the
+// values of the stored pair, hi' + lo' (fp32 bits), for the weight update.
+template <bool APPLY>
+__device__ __forceinline__ void eu_compute(uint32_t hi_s, uint32_t lo_s, int lane, float alpha, float beta,
+                                           uint32_t (&v)[EU_COLS]) {
+#pragma unroll
+    for (int k = 0; k < EU_COLS / 8; ++k) {
+        const uint32_t off = eu_off(lane, k);
+        const uint4 hv = lds128(hi_s + off), lv = lds128(lo_s + off);
+        const uint32_t h4[4] = {hv.x, hv.y, hv.z, hv.w};
+        const uint32_t l4[4] = {lv.x, lv.y, lv.z, lv.w};
+        uint32_t ho[4], lo[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x0 = bf16_bits_lo(h4[e]) + bf16_bits_lo(l4[e]);
+            const float x1 = bf16_bits_hi(h4[e]) + bf16_bits_hi(l4[e]);
+            const float y0 = alpha * __uint_as_float(v[8 * k + 2 * e]) + beta * x0;
+            const float y1 = alpha * __uint_as_float(v[8 * k + 2 * e + 1]) + beta * x1;
+            const __nv_bfloat162 hh = __floats2bfloat162_rn(y0, y1);
+            const float2 hf = __bfloat1622float2(hh);
+            const __nv_bfloat162 ll = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
+            ho[e] = *reinterpret_cast<const uint32_t*>(&hh);
+            lo[e] = *reinterpret_cast<const uint32_t*>(&ll);
+            if (APPLY) {
+                // the stored pair is the result: the weight update uses exactly it
+                v[8 * k + 2 * e] = __float_as_uint(bf16_bits_lo(ho[e]) + bf16_bits_lo(lo[e]));
+                v[8 * k + 2 * e + 1] = __float_as_uint(bf16_bits_hi(ho[e]) + bf16_bits_hi(lo[e]));
+            }
+        }
+        sts128(hi_s + off, make_uint4(ho[0], ho[1], ho[2], ho[3]));
+        sts128(lo_s + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
+    }
+}
+
 
 // ============================================================================ one-CTA kernel
 
@@ -798,45 +859,81 @@ __device__ __forceinline__ void prefetch_w_row(const GemmParams& p, const GemmGr
     }
 }
 
-// One epilogue warp of the two-CTA UPDATE kernel: X' = alpha * acc + beta * (hi + lo),
-// stored as the pair hi' = bf16(X'), lo' = bf16(X' - hi'), for the warp's 32 rows of
-// every unit of its cluster, chunk by chunk (EU_COLS columns).  Lane 0 keeps up to
-// EU_DEPTH - 1 chunks of the iterate in flight: TMA loads of the hi and lo boxes into
-// the warp's ring buffer, completing on the buffer's mbarrier.  Each lane owns one
-// row (the tcgen05.ld 32x32b layout) and reads and rewrites its row of both boxes in
-// place (swizzled, bank-conflict free); lane 0 then stores the boxes by TMA, waits
-// until the previous chunk's stores have read their buffer and reuses it for the next
-// load.  Returns false when a bounded wait gave up.
-__device__ __forceinline__ bool update_epilogue_pair(const GemmParams& p, uint32_t rank, uint32_t warp,
-                                                  uint32_t tmem_base, uint8_t* ebuf, uint64_t* ebar,
-                                                  uint64_t* tfull, uint64_t* tempty, volatile int* abort_flag,
-                                                  int cid) {
-    const uint32_t lane = threadIdx.x & 31u;
-    const int q = (int)(warp & 3u), half = (int)((warp - 2) >> 2);
+// The TMA warp of one column half of the two-CTA UPDATE epilogue (one elected
+// thread): walks the half's load chunks of every unit of its cluster in order,
+// loading chunk j + EU_DEPTH - 1 into the ring once chunk j - 1's stores have read
+// their buffer, and storing chunk j once the half's four compute warps have arrived
+// on its done barrier.  Returns false when a bounded wait gave up.
+__device__ __forceinline__ bool update_epilogue_tma(const GemmParams& p, uint32_t rank, int half, uint8_t* ebuf,
+                                                    uint64_t* efull, uint64_t* edone, int4* coord,
+                                                    volatile int* abort_flag, int cid) {
     const int u_begin = p.unit_begin[cid], u_end = p.unit_begin[cid + 1];
-    // issuer (lane 0): the next (unit, chunk) to look at and the loads issued so far
-    int iu = u_begin, ic = 0;
-    uint32_t issued = 0, consumed = 0;
-    auto issue_next = [&]() {
-        while (iu < u_end) {
-            const int4 tile = p.units[2 * iu], sk = p.units[2 * iu + 1];
-            if (ic >= eu_nchunks(sk)) { ++iu; ic = 0; continue; }
-            const EuChunk ch = eu_chunk(p, tile, sk, ic, (int)rank, q, half);
+    // next (unit, chunk) to look at, with that unit's descriptor and group shape
+    int iu = u_begin - 1, ic = 0, inch = 0, igm = 0, ign = 0;
+    int4 itile = make_int4(0, 0, 0, 0), isk = make_int4(0, 0, 0, 0);
+    // coord[b]: (group, matrix, row0, col0) of the chunk in buffer b (shared memory)
+    uint32_t issued = 0, stored = 0;
+    bool more = true, ok = true;
+    while (true) {
+        // load chunk i once the stores of chunk i - EU_DEPTH have read its buffer: after
+        // the wait below, every store but the last one has
+        while (more && issued + 1 < stored + EU_DEPTH) {
+            if (ic >= inch) {
+                if (++iu >= u_end) { more = false; break; }
+                itile = p.units[2 * iu];
+                isk = p.units[2 * iu + 1];
+                inch = eu_nchunks(isk);
+                igm = p.groups[itile.x].m;
+                ign = p.groups[itile.x].n;
+                ic = 0;
+                continue;
+            }
+            const EuChunk ch = eu_chunk(itile, isk, igm, ign, ic, (int)rank, half);
             ++ic;
             if (!ch.load) continue;
             const uint32_t b = issued % EU_DEPTH;
             uint8_t* dst = ebuf + b * EU_BUF;
             const GemmMaps& mp = p.maps[ch.g];
-            mbar_arrive_expect_tx(&ebar[b], EU_BUF);
-            tma_load_3d(dst, &mp.xe_hi[p.parity], &ebar[b], ch.col0, ch.row0, ch.mat);
-            tma_load_3d(dst + EU_BOX, &mp.xe_lo_in, &ebar[b], ch.col0, ch.row0, ch.mat);
+            coord[b] = make_int4(ch.g, ch.mat, ch.row0, ch.col0);
+            mbar_arrive_expect_tx(&efull[b], EU_BUF);
+            tma_load_3d(dst, &mp.xe_hi[p.parity], &efull[b], ch.col0, ch.row0, ch.mat);
+            tma_load_3d(dst + EU_BOX, &mp.xe_lo_in, &efull[b], ch.col0, ch.row0, ch.mat);
             ++issued;
-            return;
         }
-    };
-    if (lane == 0)
-        for (int i = 0; i < EU_DEPTH - 1; ++i) issue_next();
+        if (stored == issued) break;
+        const uint32_t b = stored % EU_DEPTH;
+        if (!mbar_wait(&edone[b], (stored / EU_DEPTH) & 1u, abort_flag, p.err, ERR_EPILOGUE)) { ok = false; break; }
+        const int4 cd = coord[b];
+        const GemmMaps& mp = p.maps[cd.x];
+        tma_store_3d(&mp.xe_hi[p.parity ^ 1], ebuf + b * EU_BUF, cd.w, cd.z, cd.y);
+        tma_store_3d(&mp.xe_lo_out, ebuf + b * EU_BUF + EU_BOX, cd.w, cd.z, cd.y);
+        bulk_commit();
+        ++stored;
+        bulk_wait_read<1>();              // every store but this one has read its buffer
+    }
+    bulk_wait_all();
+    // loads still in flight (after an abort) must land before the CTA retires
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t i = stored; i < issued; ++i)
+        while (!mbar_try_wait(&efull[i % EU_DEPTH], (i / EU_DEPTH) & 1u) && globaltimer_ns() - t0 < 100000000ull) { }
+    return ok;
+}
 
+// One compute warp of the two-CTA UPDATE epilogue: X' = alpha * acc + beta * (hi + lo),
+// stored as the pair hi' = bf16(X'), lo' = bf16(X' - hi'), for the warp's 32 rows of
+// every chunk of its column half.  Each lane owns one row (the tcgen05.ld 32x32b
+// layout) and rewrites its row of both boxes in place; the warp then arrives on the
+// chunk's done barrier for the TMA warp.  The fused weight update (last iteration)
+// follows from registers.  Returns false when a bounded wait gave up.
+__device__ __forceinline__ bool update_epilogue_compute(const GemmParams& p, uint32_t rank, uint32_t warp,
+                                                        uint32_t tmem_base, uint8_t* ebuf, uint64_t* efull,
+                                                        uint64_t* edone, uint64_t* tfull, uint64_t* tempty,
+                                                        volatile int* abort_flag, int cid) {
+    const uint32_t lane = threadIdx.x & 31u;
+    const int q = (int)(warp & 3u), half = (int)((warp - 2) >> 2);
+    const int u_begin = p.unit_begin[cid], u_end = p.unit_begin[cid + 1];
+    const int brow = q * 32 + (int)lane;             // this lane's row in the chunk boxes
+    uint32_t consumed = 0;
     bool ok = true;
     int local = 0;
     for (int u = u_begin; u < u_end && ok; ++u, ++local) {
@@ -844,10 +941,10 @@ __device__ __forceinline__ bool update_epilogue_pair(const GemmParams& p, uint32
         const int4 sk = p.units[2 * u + 1];
         const int kind = sk.z & 0xFF, nh = sk.z >> 8, slot = sk.w & 0xFFFF, nsl = sk.w >> 16;
         const GemmGroupInfo& gi = p.groups[tile.x];
+        const int gm = gi.m, gn = gi.n;
         const uint32_t acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
-        const int row_local = q * 32 + (int)lane;
-        const int row = tile.z * S2_BM + (int)rank * 128 + row_local;
+        const int row = tile.z * S2_BM + (int)rank * 128 + brow;
         if (kind != 2)
             prefetch_w_row(p, gi, tile.y, row, tile.w * S2_BN + (nh ? (nh - 1) * 128 + half * 64 : half * 128),
                            nh ? 64 : 128);
@@ -866,16 +963,16 @@ __device__ __forceinline__ bool update_epilogue_pair(const GemmParams& p, uint32
             beta *= sc;
         }
         float* sk_row = kind == 0 ? nullptr
-                      : p.sk_partial + (size_t)slot * SK_SLOT_FLOATS + ((size_t)rank * 128 + row_local) * 256;
+                      : p.sk_partial + (size_t)slot * SK_SLOT_FLOATS + ((size_t)rank * 128 + brow) * 256;
         const uint32_t tacc = tmem_base + acc * ACC_COLS + (((uint32_t)q * 32u) << 16);
         const EwSeg* sg = p.apply_mode != 0 ? &p.segs[gi.mat_base + tile.y] : nullptr;
         const int nch = (nh ? 64 : 128) / EU_COLS;
         for (int c = 0; c < nch; ++c) {
-            const EuChunk ch = eu_chunk(p, tile, sk, c, (int)rank, q, half);
+            const EuChunk ch = eu_chunk(tile, sk, gm, gn, c, (int)rank, half);
             if (kind == 2) {
                 // a later K range of a split tile: its raw partial sum goes to the slot
                 uint32_t v[EU_COLS];
-                tmem_ld_row<EU_COLS>(tacc + (uint32_t)ch.tcol, v);
+                tmem_ld_32x32b_x32(tacc + (uint32_t)ch.tcol, v);
                 tmem_ld_wait();
                 float4* dst = reinterpret_cast<float4*>(sk_row + ch.tcol);
 #pragma unroll
@@ -884,9 +981,9 @@ __device__ __forceinline__ bool update_epilogue_pair(const GemmParams& p, uint32
                                           __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
                 continue;
             }
-            if (!ch.load) continue;               // the warp's rows or columns lie outside the matrix
+            if (!ch.load) continue;               // the CTA's rows or the columns lie outside the matrix
             uint32_t v[EU_COLS];
-            tmem_ld_row<EU_COLS>(tacc + (uint32_t)ch.tcol, v);
+            tmem_ld_32x32b_x32(tacc + (uint32_t)ch.tcol, v);
             tmem_ld_wait();
             if (kind == 1) {
                 for (int sl = 0; sl < nsl; ++sl) {
@@ -902,47 +999,16 @@ __device__ __forceinline__ bool update_epilogue_pair(const GemmParams& p, uint32
                 }
             }
             const uint32_t b = consumed % EU_DEPTH;
-            ok = mbar_wait(&ebar[b], (consumed / EU_DEPTH) & 1u, abort_flag, p.err, ERR_EPILOGUE);
+            ok = mbar_wait(&efull[b], (consumed / EU_DEPTH) & 1u, abort_flag, p.err, ERR_EPILOGUE);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
-            const uint32_t hi_s = smem_u32(ebuf + b * EU_BUF), lo_s = hi_s + EU_BOX;
-            float res[EU_COLS];
-#pragma unroll
-            for (int k = 0; k < EU_COLS / 8; ++k) {
-                const uint32_t off = eu_off((int)lane, k);
-                const uint4 hv = lds128(hi_s + off), lv = lds128(lo_s + off);
-                const uint32_t h4[4] = {hv.x, hv.y, hv.z, hv.w};
-                const uint32_t l4[4] = {lv.x, lv.y, lv.z, lv.w};
-                uint32_t ho[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x0 = bf16_bits_lo(h4[e]) + bf16_bits_lo(l4[e]);
-                    const float x1 = bf16_bits_hi(h4[e]) + bf16_bits_hi(l4[e]);
-                    const float y0 = alpha * __uint_as_float(v[8 * k + 2 * e]) + beta * x0;
-                    const float y1 = alpha * __uint_as_float(v[8 * k + 2 * e + 1]) + beta * x1;
-                    const __nv_bfloat162 hh = __floats2bfloat162_rn(y0, y1);
-                    const float2 hf = __bfloat1622float2(hh);
-                    const __nv_bfloat162 ll = __floats2bfloat162_rn(y0 - hf.x, y1 - hf.y);
-                    ho[e] = *reinterpret_cast<const uint32_t*>(&hh);
-                    lo[e] = *reinterpret_cast<const uint32_t*>(&ll);
-                    // the stored pair is the result: the weight update uses exactly it
-                    res[8 * k + 2 * e] = bf16_bits_lo(ho[e]) + bf16_bits_lo(lo[e]);
-                    res[8 * k + 2 * e + 1] = bf16_bits_hi(ho[e]) + bf16_bits_hi(lo[e]);
-                }
-                sts128(hi_s + off, make_uint4(ho[0], ho[1], ho[2], ho[3]));
-                sts128(lo_s + off, make_uint4(lo[0], lo[1], lo[2], lo[3]));
-            }
+            const uint32_t hi_s = smem_u32(ebuf + b * EU_BUF) + (uint32_t)(q * 32 * EU_ROW_BYTES), lo_s = hi_s + EU_BOX;
+            if (sg != nullptr) eu_compute<true>(hi_s, lo_s, (int)lane, alpha, beta, v);
+            else eu_compute<false>(hi_s, lo_s, (int)lane, alpha, beta, v);
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                const GemmMaps& mp = p.maps[ch.g];
-                tma_store_3d(&mp.xe_hi[p.parity ^ 1], ebuf + b * EU_BUF, ch.col0, ch.row0, ch.mat);
-                tma_store_3d(&mp.xe_lo_out, ebuf + b * EU_BUF + EU_BOX, ch.col0, ch.row0, ch.mat);
-                bulk_commit();
-                bulk_wait_read<1>();          // the previous chunk's buffer is free again
-                issue_next();
-            }
+            if (lane == 0) mbar_arrive(&edone[b]);
             ++consumed;
-            if (sg != nullptr && row < gi.m) apply_row<EU_COLS>(p, gi, *sg, row, ch.col0, res);
+            if (sg != nullptr && row < gm) apply_row<EU_COLS>(p, gi, *sg, row, ch.col0, v);
         }
         if (!ok) break;
         tc_fence_before();
@@ -958,21 +1024,13 @@ __device__ __forceinline__ bool update_epilogue_pair(const GemmParams& p, uint32
             mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
         }
     }
-    if (lane == 0) {
-        bulk_wait_all();
-        // loads still in flight (after an abort) must land before the CTA retires
-        const uint64_t t0 = globaltimer_ns();
-        for (uint32_t i = consumed; i < issued; ++i)
-            while (!mbar_try_wait(&ebar[i % EU_DEPTH], (i / EU_DEPTH) & 1u) && globaltimer_ns() - t0 < 100000000ull) { }
-    }
-    __syncwarp();
     return ok;
 }
 
 // ============================================================================ two-CTA kernel
 
 template <int MODE>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NUM_THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(s2_threads(MODE), 1)
 ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
     constexpr int STAGES = s2_stages(MODE);
     extern __shared__ uint8_t smem_raw[];
@@ -986,8 +1044,11 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
     uint64_t* ebar = drain + 1;                            // UPDATE: EU_DEPTH per epilogue warp
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + (MODE == MODE_UPDATE ? NUM_EPI_WARPS * EU_DEPTH : 0));
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + (MODE == MODE_UPDATE ? 4 * EU_DEPTH : 0));
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    // UPDATE: 2 x EU_DEPTH chunk coordinates after the TMEM address and the abort flag,
+    // rounded up to a 16-byte boundary
+    int4* ecoord = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(tmem_slot + 2) + 15) & ~uintptr_t(15));
 
     const uint32_t warp = warp_id();
     const uint32_t lane = threadIdx.x & 31u;
@@ -1005,7 +1066,11 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
         }
         mbar_init(drain, 1);
         if (MODE == MODE_UPDATE)
-            for (int i = 0; i < NUM_EPI_WARPS * EU_DEPTH; ++i) mbar_init(&ebar[i], 1);
+            for (int h = 0; h < 2; ++h)
+                for (int i = 0; i < EU_DEPTH; ++i) {
+                    mbar_init(&ebar[h * 2 * EU_DEPTH + i], 1);                  // full: the TMA warp's expect_tx
+                    mbar_init(&ebar[h * 2 * EU_DEPTH + EU_DEPTH + i], 4);       // done: the half's compute warps
+                }
         *abort_flag = 0;
         fence_barrier_init();
     }
@@ -1024,10 +1089,15 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
         if (elect_one()) {
             uint32_t stage = 0, phase = 0;
             bool ok = true;
-            const int u_end = p.unit_begin[cid + 1];
-            for (int u = p.unit_begin[cid]; u < u_end && ok; ++u) {
-                const int4 tile = p.units[2 * u];
-                const int4 sk = p.units[2 * u + 1];
+            const int u_begin = p.unit_begin[cid], u_end = p.unit_begin[cid + 1];
+            // the next unit's descriptor is loaded one unit ahead: its latency hides
+            // behind the current unit's loads instead of stalling the ring
+            int4 tile_next = make_int4(0, 0, 0, 0), sk_next = make_int4(0, 0, 0, 0);
+            if (u_begin < u_end) { tile_next = p.units[2 * u_begin]; sk_next = p.units[2 * u_begin + 1]; }
+            for (int u = u_begin; u < u_end && ok; ++u) {
+                const int4 tile = tile_next;
+                const int4 sk = sk_next;
+                if (u + 1 < u_end) { tile_next = p.units[2 * u + 2]; sk_next = p.units[2 * u + 3]; }
                 const void *mapA, *mapB;
                 operand_maps<MODE>(p, tile.x, mapA, mapB);
                 const int nh = sk.z >> 8;                              // 0: full tile, 1/2: column half
@@ -1064,9 +1134,13 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
             uint32_t stage = 0, phase = 0;
             int local = 0;
             bool ok = true;
-            const int u_end = p.unit_begin[cid + 1];
-            for (int u = p.unit_begin[cid]; u < u_end && ok; ++u, ++local) {
-                const int4 sk = p.units[2 * u + 1];
+            const int u_begin = p.unit_begin[cid], u_end = p.unit_begin[cid + 1];
+            // loaded one unit ahead, so that the tensor pipe does not drain while the
+            // next unit's K range is fetched
+            int4 sk_next = u_begin < u_end ? p.units[2 * u_begin + 1] : make_int4(0, 0, 0, 0);
+            for (int u = u_begin; u < u_end && ok; ++u, ++local) {
+                const int4 sk = sk_next;
+                if (u + 1 < u_end) sk_next = p.units[2 * u + 3];
                 const uint32_t idesc = (sk.z >> 8) ? idesc_half : idesc_full;
                 const uint32_t acc = local & 1;
                 const uint32_t acc_phase = (local >> 1) & 1;
@@ -1103,8 +1177,17 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
             }
         }
     } else if (MODE == MODE_UPDATE) {
-        update_epilogue_pair(p, rank, warp, tmem_base, sE + (warp - 2) * (EU_DEPTH * EU_BUF),
-                             ebar + (warp - 2) * EU_DEPTH, tfull, tempty, abort_flag, cid);
+        // ring of column half h: buffers sE + h * EU_DEPTH * EU_BUF, barriers
+        // ebar[4h * ...]: EU_DEPTH full (TMA loads), then EU_DEPTH done (compute warps)
+        if (warp < 2 + NUM_EPI_WARPS) {
+            const int h = (int)((warp - 2) >> 2);
+            update_epilogue_compute(p, rank, warp, tmem_base, sE + h * (EU_DEPTH * EU_BUF), ebar + h * 2 * EU_DEPTH,
+                                    ebar + h * 2 * EU_DEPTH + EU_DEPTH, tfull, tempty, abort_flag, cid);
+        } else if (elect_one()) {
+            const int h = (int)(warp - 2 - NUM_EPI_WARPS);
+            update_epilogue_tma(p, rank, h, sE + h * (EU_DEPTH * EU_BUF), ebar + h * 2 * EU_DEPTH,
+                                ebar + h * 2 * EU_DEPTH + EU_DEPTH, ecoord + h * EU_DEPTH, abort_flag, cid);
+        }
     } else {
         const uint32_t q = warp & 3u;
         const uint32_t half = (warp - 2) >> 2;
@@ -1167,6 +1250,7 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
 size_t tc_gemm_smem_bytes(int pair) { return pair ? S2_SMEM : S1_SMEM; }
 size_t tc_gemm_smem_bytes_mode(int mode, int pair) { return pair ? (size_t)s2_smem(mode) : (size_t)S1_SMEM; }
 int tc_gemm_epi_cols() { return EU_COLS; }
+int tc_gemm_epi_rows() { return EU_ROWS; }
 int tc_gemm_threads() { return NUM_THREADS; }
 int tc_gemm_tile_m(int pair) { return pair ? S2_BM : S1_BM; }
 int tc_gemm_tile_n(int pair) { return pair ? S2_BN : S1_BN; }
@@ -1189,7 +1273,7 @@ cudaError_t tc_gemm_max_clusters(int* n) {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(2, 1, 1);
-    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+    cfg.blockDim = dim3(NUM_THREADS_U, 1, 1);
     cfg.dynamicSmemBytes = S2U_SMEM;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -1197,6 +1281,7 @@ cudaError_t tc_gemm_max_clusters(int* n) {
     cudaError_t e = cudaOccupancyMaxActiveClusters(&nu, ns_gemm_tc2_kernel<MODE_UPDATE>, &cfg);
     if (e != cudaSuccess) return e;
     cfg.dynamicSmemBytes = S2_SMEM;
+    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
     e = cudaOccupancyMaxActiveClusters(&ng, ns_gemm_tc2_kernel<MODE_GRAM>, &cfg);
     *n = nu < ng ? nu : ng;
     return e;
@@ -1209,7 +1294,7 @@ cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cu
         switch (mode) {
             case MODE_GRAM: return launch_pdl(ns_gemm_tc2_kernel<MODE_GRAM>, g, b, S2_SMEM, s, p);
             case MODE_POLY: return launch_pdl(ns_gemm_tc2_kernel<MODE_POLY>, g, b, S2_SMEM, s, p);
-            default: return launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE>, g, b, S2U_SMEM, s, p);
+            default: return launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE>, g, dim3(NUM_THREADS_U), S2U_SMEM, s, p);
         }
     }
     switch (mode) {

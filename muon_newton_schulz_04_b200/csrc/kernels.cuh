@@ -50,6 +50,7 @@ struct EwSeg {
     int apply_count;
     int mat;              // global matrix index (norm / scale arrays)
     float update_scale;   // per-shape scale s of the update
+    int out_bf16;         // copy-out only: `w` receives O as bf16 instead of fp32
 };
 
 struct alignas(64) GemmMaps {
@@ -57,7 +58,7 @@ struct alignas(64) GemmMaps {
     CUtensorMap xb_mn[2];  // X operand, box {64, 64}: X as an N-contiguous operand
     CUtensorMap a;         // A, box {64, 128}
     CUtensorMap p;         // P, box {64, 128}
-    // UPDATE epilogue of the two-CTA kernel: 32 x 32 boxes of the iterate, 64-byte
+    // UPDATE epilogue of the two-CTA kernel: 128 x 32 boxes of the iterate, 64-byte
     // swizzle, loaded into and stored from shared memory (hi in / hi out follow the
     // ping-pong parity; lo in and lo out are the same array in a step)
     CUtensorMap xe_hi[2];
@@ -108,8 +109,9 @@ constexpr int SK_SLOT_FLOATS = 2 * 128 * 256;
 // pair = 0: the one-CTA kernel (128 x 256 tiles).
 size_t tc_gemm_smem_bytes(int pair);
 size_t tc_gemm_smem_bytes_mode(int mode, int pair);
-// columns of one box of the two-CTA UPDATE epilogue (16 or 32; boxes are 32 rows)
+// box of the two-CTA UPDATE epilogue: rows x columns (128 x 32 bf16)
 int tc_gemm_epi_cols();
+int tc_gemm_epi_rows();
 int tc_gemm_threads();
 int tc_gemm_tile_m(int pair);
 int tc_gemm_tile_n(int pair);

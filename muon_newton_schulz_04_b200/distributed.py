@@ -1,19 +1,28 @@
-"""Matrix-sharded Muon over data-parallel ranks (one process per GPU).
+"""Muon over data-parallel ranks (one process per GPU), two ways of sharding it.
 
 Every matrix's step is independent ("Muon: An optimizer for hidden layers in
-neural networks", section 4 defines the update per matrix), so under data
-parallelism -- every rank holds the same, already averaged gradients -- rank r
-steps only the matrices it owns and keeps only their momentum buffers (the
-optimizer-state sharding of the Moonlight result's Distributed Muon, whole
-matrices instead of row slices, so no gradient needs gathering).  One collective
-then hands every rank the updated weights: each rank packs its updated matrices
-into one flat buffer, and a single all-gather (NCCL over NVLink on GPUs, gloo in
-the CPU tests) delivers all shards.
+neural networks", section 4 defines the update per matrix), and under data
+parallelism every rank holds the same, already averaged gradients.
 
-Ownership is decided once by longest-processing-time-first on the nominal
-Newton-Schulz FLOPs 5 (4 m^2 n + 2 m^3) of each matrix, so ranks finish at about
-the same time.  All Muon arithmetic runs in the CUDA library; this module only
-partitions, packs and calls the collective.
+ShardedMuon -- whole matrices are owned by ranks (longest-processing-time-first
+  on the nominal Newton-Schulz FLOPs 5 (4 m^2 n + 2 m^3), so ranks finish at
+  about the same time).  A rank keeps only its matrices' momentum, computes only
+  their update directions O (muon_step_direction), writes them in bf16 into one
+  packed buffer, and a single all-gather hands every rank every O; each rank then
+  applies every O to its copy of the weights (muon_apply).  All ranks apply the
+  same bf16 O with the same kernel, so their weights stay bitwise identical, and
+  the exchange moves 2 bytes per weight instead of the 4 of an fp32 weight.
+
+Zero1Muon -- the optimizer-state sharding of the Moonlight result's Distributed
+  Muon ("关键实验/定理", result 2): rank r keeps the momentum rows [r0, r1) of every
+  matrix, updates them from its rows of the gradient, and the ranks all-gather the
+  rows of the Nesterov direction U so that each holds every full U; each rank then
+  orthogonalises every full matrix (muon_orthogonalize; the same work on every
+  rank), updates its own rows of W and the ranks all-gather the updated rows.
+
+All Muon arithmetic runs in the CUDA library by default; this module partitions,
+packs and calls the collectives.  The CPU tests substitute the fp64 oracle for
+the per-rank functions to check the host logic with gloo ranks.
 """
 from __future__ import annotations
 
@@ -44,61 +53,216 @@ def lpt_partition(costs: Sequence[float], world: int) -> List[List[int]]:
     return [sorted(p) for p in parts]
 
 
+def row_slices(rows: int, world: int) -> List[Tuple[int, int]]:
+    """Rows [r0, r1) of each rank: as even as possible, the first `rows % world`
+    ranks one row longer."""
+    base, extra = divmod(rows, world)
+    out, r0 = [], 0
+    for r in range(world):
+        r1 = r0 + base + (1 if r < extra else 0)
+        out.append((r0, r1))
+        r0 = r1
+    return out
+
+
+def _pad8(n: int) -> int:
+    return (n + 7) // 8 * 8         # 16-byte aligned bf16 / 32-byte aligned fp32 slots
+
+
+def _by_shape(*lists):
+    """Zips same-index items and groups them by the shape of the first list."""
+    groups = {}
+    for items in zip(*lists):
+        groups.setdefault(tuple(items[0].shape), []).append(items)
+    return [tuple(list(x) for x in zip(*v)) for v in groups.values()]
+
+
+def _world_rank(group):
+    if dist.is_available() and dist.is_initialized():
+        return dist.get_world_size(group), dist.get_rank(group)
+    return 1, 0
+
+
 class ShardedMuon:
     """Muon over a list of 2D weights, sharded by whole matrices across ranks.
 
     shapes: (rows, cols) of every matrix, identical on all ranks.
-    local_step(W_own, G_own, B_own): runs the Muon step of the rank's own matrices
-    in place (by default the CUDA library's muon_step through the binding).
+    direction_fn(G_own, B_own, O_own): updates B_own in place and writes the update
+      direction of each own matrix into O_own (views of the packed send buffer, in
+      `payload_dtype`); by default muon_step_direction.
+    apply_fn(W, O): W <- W - lr*wd*W - lr*s*O for every matrix; by default muon_apply.
     """
 
     def __init__(self, shapes: Sequence[Tuple[int, int]], cfg=None, group=None, device=None,
-                 local_step: Optional[Callable] = None):
+                 direction_fn: Optional[Callable] = None, apply_fn: Optional[Callable] = None,
+                 payload_dtype=torch.bfloat16):
         self.shapes = [tuple(s) for s in shapes]
         self.group = group
-        self.world = dist.get_world_size(group) if dist.is_initialized() else 1
-        self.rank = dist.get_rank(group) if dist.is_initialized() else 0
+        self.world, self.rank = _world_rank(group)
+        self.payload_dtype = payload_dtype
         steps = getattr(cfg, "ns_steps", 5) if cfg is not None else 5
         self.parts = lpt_partition([ns_flops(r, c, steps) for (r, c) in self.shapes], self.world)
         self.own = self.parts[self.rank]
-        self.shard_elems = [sum(self.shapes[k][0] * self.shapes[k][1] for k in p) for p in self.parts]
-        self.max_elems = max(self.shard_elems) if self.shard_elems else 0
-        if local_step is None:
-            from . import Group, Muon
+        # packed layout: rank r's matrices in increasing index order, each slot padded
+        self.offset = {}
+        sizes = []
+        for part in self.parts:
+            off = 0
+            for k in part:
+                self.offset[k] = off
+                off += _pad8(self.shapes[k][0] * self.shapes[k][1])
+            sizes.append(off)
+        self.max_elems = max(sizes) if sizes else 0
+        if direction_fn is None or apply_fn is None:
+            from . import Muon
             opt = Muon(cfg, device=0 if device is None else device)
-
-            def local_step(W, G, B):
-                groups = {}
-                for w, g, b in zip(W, G, B):
-                    groups.setdefault(tuple(w.shape), []).append((w, g, b))
-                opt.step([Group(W=[x[0] for x in v], G=[x[1] for x in v], B=[x[2] for x in v])
-                          for v in groups.values()])
             self._opt = opt
-        self.local_step = local_step
+            if direction_fn is None:
+                def direction_fn(G, B, O):
+                    opt.step_direction(_by_shape(G, B, O))
+            if apply_fn is None:
+                def apply_fn(W, O):
+                    opt.apply(_by_shape(W, O))
+        self.direction_fn, self.apply_fn = direction_fn, apply_fn
+        self._send = self._recv = None
 
     def new_momentum(self, like: Sequence[torch.Tensor]) -> List[torch.Tensor]:
         """Zeroed fp32 momentum buffers for the rank's own matrices only."""
         return [torch.zeros_like(like[k], dtype=torch.float32) for k in self.own]
 
+    def _views(self, buf, r, ks):
+        base = r * self.max_elems
+        return [buf[base + self.offset[k]: base + self.offset[k] + self.shapes[k][0] * self.shapes[k][1]]
+                .view(self.shapes[k]) for k in ks]
+
     def step(self, W: Sequence[torch.Tensor], G: Sequence[torch.Tensor], B_own: Sequence[torch.Tensor]) -> None:
-        """One step: update the own matrices, then all-gather every shard into W."""
-        self.local_step([W[k] for k in self.own], [G[k] for k in self.own], list(B_own))
+        """One step: own directions into the packed buffer, one all-gather, then every
+        rank applies every matrix's O to its weights."""
+        dev = W[0].device
+        if self._send is None or self._send.device != dev:
+            self._send = torch.zeros(max(self.max_elems, 1), dtype=self.payload_dtype, device=dev)
+            self._recv = (self._send if self.world == 1 else
+                          torch.zeros(self.world * max(self.max_elems, 1), dtype=self.payload_dtype, device=dev))
+        if self.own:
+            self.direction_fn([G[k] for k in self.own], list(B_own), self._views(self._send, 0, self.own))
+        if self.world > 1:
+            dist.all_gather_into_tensor(self._recv, self._send, group=self.group)
+        ks, Os = [], []
+        for r, part in enumerate(self.parts):
+            ks += part
+            Os += self._views(self._recv, r if self.world > 1 else 0, part)
+        if ks:
+            self.apply_fn([W[k] for k in ks], Os)
+
+
+class Zero1Muon:
+    """Muon with row-sliced optimizer state (ZeRO-1 style Distributed Muon).
+
+    shapes: (rows, cols) of every matrix, identical on all ranks.
+    momentum_fn(G_rows, B_rows, U_rows): B <- mu*B + G in place and U = the Nesterov
+      direction, for the rank's row slices (by default the library's momentum
+      kernel, muon_momentum_norm_noalloc, one slice at a time);
+    ortho_fn(U, O): O = NS(U / (||U||_F + eps)) for full matrices (muon_orthogonalize);
+    apply_fn(W_rows, O_rows): the update of the own rows (muon_apply).
+    U is gathered in `u_dtype` (fp32 by default; the CPU tests use fp64).
+    """
+
+    def __init__(self, shapes: Sequence[Tuple[int, int]], cfg=None, group=None, device=None,
+                 momentum_fn: Optional[Callable] = None, ortho_fn: Optional[Callable] = None,
+                 apply_fn: Optional[Callable] = None, u_dtype=torch.float32):
+        self.shapes = [tuple(s) for s in shapes]
+        self.group = group
+        self.world, self.rank = _world_rank(group)
+        self.u_dtype = u_dtype
+        self.slices = [row_slices(r, self.world) for (r, _) in self.shapes]
+        # packed layout of one rank's rows of every matrix (padded to the largest rank)
+        self.offset = []
+        sizes = [0] * self.world
+        for k, (r, c) in enumerate(self.shapes):
+            offs = []
+            for rk in range(self.world):
+                r0, r1 = self.slices[k][rk]
+                offs.append(sizes[rk])
+                sizes[rk] += _pad8((r1 - r0) * c)
+            self.offset.append(offs)
+        self.max_elems = max(sizes) if sizes else 0
+        if momentum_fn is None or ortho_fn is None or apply_fn is None:
+            from . import Muon, momentum_norm_noalloc
+            opt = Muon(cfg, device=0 if device is None else device)
+            self._opt = opt
+            mu = float(opt.cfg.momentum)
+            nesterov = bool(opt.cfg.nesterov)
+            if momentum_fn is None:
+                norm = torch.empty(1, dtype=torch.float32, device=torch.device("cuda", opt.device))
+
+                def momentum_fn(G, B, U):
+                    for g, b, u in zip(G, B, U):
+                        if b.numel():
+                            momentum_norm_noalloc(g, b, norm, U_out=u, momentum=mu, nesterov=nesterov)
+            if ortho_fn is None:
+                def ortho_fn(U, O):
+                    opt.orthogonalize([(list(a), list(b)) for (a, b) in _by_shape(U, O)])
+            if apply_fn is None:
+                def apply_fn(W, O):
+                    keep = [(w, o) for w, o in zip(W, O) if w.numel()]
+                    if keep:
+                        opt.apply(_by_shape([w for w, _ in keep], [o for _, o in keep]))
+        self.momentum_fn, self.ortho_fn, self.apply_fn = momentum_fn, ortho_fn, apply_fn
+        self._bufs = None
+
+    def new_momentum(self, like: Sequence[torch.Tensor]) -> List[torch.Tensor]:
+        """Zeroed fp32 momentum rows [r0, r1) of every matrix for this rank."""
+        out = []
+        for k, w in enumerate(like):
+            r0, r1 = self.slices[k][self.rank]
+            out.append(torch.zeros((r1 - r0, w.shape[1]), dtype=torch.float32, device=w.device))
+        return out
+
+    def _rows(self, buf, rk, k, slot):
+        """Rank rk's rows of matrix k in a packed buffer: in slot `slot` of a gathered
+        buffer (slot = rk), or at the start of a send buffer (slot = 0)."""
+        r0, r1 = self.slices[k][rk]
+        c = self.shapes[k][1]
+        base = slot * self.max_elems + self.offset[k][rk]
+        return buf[base: base + (r1 - r0) * c].view(r1 - r0, c)
+
+    def step(self, W: Sequence[torch.Tensor], G: Sequence[torch.Tensor], B_own: Sequence[torch.Tensor]) -> None:
+        dev = W[0].device
+        n = max(self.max_elems, 1)
+        if self._bufs is None or self._bufs[0].device != dev:
+            u_send = torch.zeros(n, dtype=self.u_dtype, device=dev)
+            u_recv = u_send if self.world == 1 else torch.zeros(self.world * n, dtype=self.u_dtype, device=dev)
+            w_send = torch.zeros(n, dtype=W[0].dtype, device=dev)
+            w_recv = w_send if self.world == 1 else torch.zeros(self.world * n, dtype=W[0].dtype, device=dev)
+            self._bufs = (u_send, u_recv, w_send, w_recv)
+        u_send, u_recv, w_send, w_recv = self._bufs
+        K = len(self.shapes)
+        me = self.rank
+        # 1. momentum and direction on the own rows
+        G_rows = [G[k][self.slices[k][me][0]: self.slices[k][me][1]] for k in range(K)]
+        U_rows = [self._rows(u_send, me, k, 0) for k in range(K)]
+        self.momentum_fn(G_rows, list(B_own), U_rows)
+        # 2. every rank gets every full U
+        if self.world > 1:
+            dist.all_gather_into_tensor(u_recv, u_send, group=self.group)
+        U_full = []
+        for k in range(K):
+            parts = [self._rows(u_recv, rk, k, rk) for rk in range(self.world)]
+            U_full.append(parts[0] if self.world == 1 else torch.cat(parts, 0))
+        # 3. orthogonalise every full matrix (the same work on every rank)
+        O_full = [torch.empty(s, dtype=self.u_dtype, device=dev) for s in self.shapes]
+        self.ortho_fn(U_full, O_full)
+        # 4. update the own rows of W, then hand every rank every updated row
+        W_rows = [W[k][self.slices[k][me][0]: self.slices[k][me][1]] for k in range(K)]
+        O_rows = [O_full[k][self.slices[k][me][0]: self.slices[k][me][1]] for k in range(K)]
+        self.apply_fn(W_rows, O_rows)
         if self.world == 1:
             return
-        dev = W[0].device
-        send = torch.zeros(self.max_elems, dtype=W[0].dtype, device=dev)
-        off = 0
-        for k in self.own:
-            n = W[k].numel()
-            send[off:off + n].copy_(W[k].reshape(-1))
-            off += n
-        recv = torch.empty(self.world * self.max_elems, dtype=W[0].dtype, device=dev)
-        dist.all_gather_into_tensor(recv, send, group=self.group)
-        for r, part in enumerate(self.parts):
-            if r == self.rank:
-                continue
-            off = r * self.max_elems
-            for k in part:
-                n = W[k].numel()
-                W[k].copy_(recv[off:off + n].view_as(W[k]))
-                off += n
+        for k in range(K):
+            self._rows(w_send, me, k, 0).copy_(W_rows[k])
+        dist.all_gather_into_tensor(w_recv, w_send, group=self.group)
+        for k in range(K):
+            for rk in range(self.world):
+                r0, r1 = self.slices[k][rk]
+                if rk != me and r1 > r0:
+                    W[k][r0:r1].copy_(self._rows(w_recv, rk, k, rk))

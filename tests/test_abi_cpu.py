@@ -355,3 +355,11 @@ def test_binding_refuses_tensors_of_another_device():
         mb.momentum_norm_noalloc(on0(bf), on0(), n1)
     with pytest.raises(ValueError, match="cuda:1"):
         mb.momentum_norm_noalloc(on0(bf), on0(), _FakeCudaTensor((1,), f32, 0), U_out=on1())
+
+
+def test_direction_and_apply_reject_a_null_handle():
+    """The two entry points of the sharded step refuse a NULL handle on the host
+    (their other argument checks run on a handle and are tested on the GPU)."""
+    L = mb.lib()
+    assert L.muon_step_direction(None, None, 0, None) == mb.MUON_ERR_INVALID
+    assert L.muon_apply(None, None, 0, None) == mb.MUON_ERR_INVALID
