@@ -392,11 +392,15 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
         for (int z = 0; z < d.count; ++z, ++mat) {
             EwSeg sg{};
             sg.rows = d.rows; sg.cols = d.cols; sg.ldn = d.ldn; sg.transposed = d.transposed;
-            int nb;
-            if (d.transposed) nb = ((d.rows + EW_TILE - 1) / EW_TILE) * ((d.cols + EW_TILE - 1) / EW_TILE);
-            else nb = (int)(((long long)d.rows * d.cols + EW_FLAT_ELEMS - 1) / EW_FLAT_ELEMS);
+            int nb, na;
+            if (d.transposed) {
+                nb = ((d.rows + MT_ROWS - 1) / MT_ROWS) * ((d.cols + MT_COLS - 1) / MT_COLS);
+                na = ((d.rows + EW_TILE - 1) / EW_TILE) * ((d.cols + EW_TILE - 1) / EW_TILE);
+            } else {
+                nb = na = (int)(((long long)d.rows * d.cols + EW_FLAT_ELEMS - 1) / EW_FLAT_ELEMS);
+            }
             sg.blk_begin = k1; sg.blk_count = nb; k1 += nb;
-            sg.apply_begin = k7; sg.apply_count = nb; k7 += nb;
+            sg.apply_begin = k7; sg.apply_count = na; k7 += na;
             sg.mat = mat;
             P.segs.push_back(sg);
         }

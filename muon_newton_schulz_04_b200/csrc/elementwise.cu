@@ -109,7 +109,7 @@ __global__ void __launch_bounds__(EW_THREADS, EW_MIN_BLOCKS) momentum_norm_kerne
                                                                   int nesterov, int bf16_operand,
                                                                   int* __restrict__ counters, float eps,
                                                                   float* __restrict__ norms, float* __restrict__ scale) {
-    __shared__ float tile[EW_TILE][EW_TILE + 1];
+    __shared__ float tile_t[MT_COLS][MT_ROWS + 1];     // transposed tile of a tall matrix
     __shared__ double red[EW_THREADS / 32];
     pdl_trigger();
     pdl_wait();
@@ -201,105 +201,115 @@ __global__ void __launch_bounds__(EW_THREADS, EW_MIN_BLOCKS) momentum_norm_kerne
             }
         }
     } else {
-        // tall matrix: X = U^T.  Tile of U rows [i0, i0+64) x cols [j0, j0+64).
-        const int tiles_c = (sg.cols + EW_TILE - 1) / EW_TILE;
-        const int i0 = (lb / tiles_c) * EW_TILE, j0 = (lb % tiles_c) * EW_TILE;
+        // tall matrix: X = U^T.  Tile of U rows [i0, i0 + MT_ROWS) x cols [j0, j0 + MT_COLS):
+        // 8192 elements, the flat path's block size.  U is read and B written along W's
+        // rows; X0 is written along X's rows from the shared tile tr[j][i] (row stride
+        // MT_ROWS + 1), so both sides of the transpose stay coalesced.
+        const int tiles_c = (sg.cols + MT_COLS - 1) / MT_COLS;
+        const int i0 = (lb / tiles_c) * MT_ROWS, j0 = (lb % tiles_c) * MT_COLS;
         if (sg.vec && sg.b != nullptr) {
-            // 16 x 16 threads, each on 4 consecutive columns of 4 rows (r, r+16, r+32,
-            // r+48): every G and B load of the thread is issued before any arithmetic.
-            // cols % 8 == 0, so a 4-column group is either wholly inside or outside.
-            const int c4 = threadIdx.x & 15, r = threadIdx.x >> 4;
-            const int j = j0 + 4 * c4;
-            constexpr int RSTEPS = EW_TILE / 16;
-            uint4 graw[RSTEPS];
-            float4 braw[RSTEPS];
+            // thread (cg, r): columns j0 + 8cg .. +7 of rows i0 + r + 16p, p = 0..3, two
+            // rows' loads in flight before any arithmetic (cols % 8 == 0: a group of 8
+            // columns lies wholly inside the matrix or wholly outside)
+            const int cg = threadIdx.x & 15, r = threadIdx.x >> 4;
+            const int j = j0 + 8 * cg;
 #pragma unroll
-            for (int k = 0; k < RSTEPS; ++k) {
-                const int i = i0 + r + 16 * k;
-                if (i >= sg.rows || j >= sg.cols) continue;
-                const size_t e = (size_t)i * sg.cols + j;
-                if (sg.g_bf16) {
-                    const uint2 v = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(sg.g) + e);
-                    graw[k] = make_uint4(v.x, v.y, 0u, 0u);
-                } else {
-                    graw[k] = *reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(sg.g) + e);
-                }
-                braw[k] = *reinterpret_cast<const float4*>(sg.b + e);
-            }
+            for (int p0 = 0; p0 < MT_ROWS / 16; p0 += 2) {
+                uint4 graw[2][2];
+                float4 braw[2][2];
 #pragma unroll
-            for (int k = 0; k < RSTEPS; ++k) {
-                const int i = i0 + r + 16 * k;
-                float u[4] = {0.f, 0.f, 0.f, 0.f};
-                if (i < sg.rows && j < sg.cols) {
-                    float g[4];
+                for (int pp = 0; pp < 2; ++pp) {
+                    const int i = i0 + r + 16 * (p0 + pp);
+                    if (i >= sg.rows || j >= sg.cols) continue;
+                    const size_t e = (size_t)i * sg.cols + j;
                     if (sg.g_bf16) {
-                        g[0] = __uint_as_float(graw[k].x << 16);
-                        g[1] = __uint_as_float(graw[k].x & 0xFFFF0000u);
-                        g[2] = __uint_as_float(graw[k].y << 16);
-                        g[3] = __uint_as_float(graw[k].y & 0xFFFF0000u);
+                        graw[pp][0] = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(sg.g) + e);
                     } else {
-                        g[0] = __uint_as_float(graw[k].x); g[1] = __uint_as_float(graw[k].y);
-                        g[2] = __uint_as_float(graw[k].z); g[3] = __uint_as_float(graw[k].w);
+                        graw[pp][0] = *reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(sg.g) + e);
+                        graw[pp][1] = *reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(sg.g) + e + 4);
                     }
-                    float b[4] = {braw[k].x, braw[k].y, braw[k].z, braw[k].w};
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        b[q] = fmaf(mu, b[q], g[q]);
-                        u[q] = nesterov ? fmaf(mu, b[q], g[q]) : b[q];
-                        acc += (double)u[q] * (double)u[q];
-                    }
-                    *reinterpret_cast<float4*>(sg.b + (size_t)i * sg.cols + j) = make_float4(b[0], b[1], b[2], b[3]);
+                    const float4* bp = reinterpret_cast<const float4*>(sg.b + e);
+                    braw[pp][0] = bp[0];
+                    braw[pp][1] = bp[1];
                 }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) tile[r + 16 * k][4 * c4 + q] = u[q];
-            }
-            __syncthreads();
-            // X[jx][i0 + 4*c4 .. +3] = U[i][jx]: 4 consecutive elements of an X row per thread
-            const int ix = i0 + 4 * c4;
+                for (int pp = 0; pp < 2; ++pp) {
+                    const int ir = r + 16 * (p0 + pp), i = i0 + ir;
+                    float u[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+                    if (i < sg.rows && j < sg.cols) {
+                        float g[8];
+                        if (sg.g_bf16) {
+                            const uint32_t w[4] = {graw[pp][0].x, graw[pp][0].y, graw[pp][0].z, graw[pp][0].w};
 #pragma unroll
-            for (int k = 0; k < RSTEPS; ++k) {
-                const int jj = r + 16 * k, jx = j0 + jj;
-                if (jx >= sg.cols || ix >= sg.rows) continue;
-                float u[4];
+                            for (int q = 0; q < 4; ++q) {
+                                g[2 * q] = __uint_as_float(w[q] << 16);
+                                g[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+                            }
+                        } else {
+                            const uint32_t w[8] = {graw[pp][0].x, graw[pp][0].y, graw[pp][0].z, graw[pp][0].w,
+                                                   graw[pp][1].x, graw[pp][1].y, graw[pp][1].z, graw[pp][1].w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) u[q] = tile[4 * c4 + q][jj];
-                const size_t xo = (size_t)jx * sg.ldn + ix;
-                if (ix + 3 < sg.rows) {
-                    if (bf16_operand) {
-                        uint32_t hw[2], lw[2];
-                        split_bf16x2(u[0], u[1], hw[0], lw[0]);
-                        split_bf16x2(u[2], u[3], hw[1], lw[1]);
-                        *reinterpret_cast<uint2*>(sg.xhi0 + xo) = make_uint2(hw[0], hw[1]);
-                        *reinterpret_cast<uint2*>(sg.xlo0 + xo) = make_uint2(lw[0], lw[1]);
-                    } else {
-                        *reinterpret_cast<float4*>(sg.xf0 + xo) = make_float4(u[0], u[1], u[2], u[3]);
+                            for (int q = 0; q < 8; ++q) g[q] = __uint_as_float(w[q]);
+                        }
+                        float bb[8] = {braw[pp][0].x, braw[pp][0].y, braw[pp][0].z, braw[pp][0].w,
+                                       braw[pp][1].x, braw[pp][1].y, braw[pp][1].z, braw[pp][1].w};
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) {
+                            bb[q] = fmaf(mu, bb[q], g[q]);
+                            u[q] = nesterov ? fmaf(mu, bb[q], g[q]) : bb[q];
+                            acc += (double)u[q] * (double)u[q];
+                        }
+                        float4* bp = reinterpret_cast<float4*>(sg.b + (size_t)i * sg.cols + j);
+                        bp[0] = make_float4(bb[0], bb[1], bb[2], bb[3]);
+                        bp[1] = make_float4(bb[4], bb[5], bb[6], bb[7]);
                     }
-                } else {
-                    for (int q = 0; ix + q < sg.rows; ++q) store_x0(sg, xo + q, u[q], bf16_operand);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) tile_t[8 * cg + q][ir] = u[q];
                 }
             }
         } else {
-            const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;     // 64 x 4
-#pragma unroll 4
-            for (int ii = ty; ii < EW_TILE; ii += 4) {
-                const int i = i0 + ii, j = j0 + tx;
+            // consecutive threads take consecutive columns of a row of U
+            for (int e = threadIdx.x; e < MT_ROWS * MT_COLS; e += EW_THREADS) {
+                const int ii = e / MT_COLS, jj = e % MT_COLS;
+                const int i = i0 + ii, j = j0 + jj;
                 float u = 0.f;
                 if (i < sg.rows && j < sg.cols) {
-                    const size_t e = (size_t)i * sg.cols + j;
-                    u = direction(load_g(sg.g, e, sg.g_bf16), sg.b ? sg.b + e : nullptr, mu, nesterov);
+                    const size_t ge = (size_t)i * sg.cols + j;
+                    u = direction(load_g(sg.g, ge, sg.g_bf16), sg.b ? sg.b + ge : nullptr, mu, nesterov);
                     acc += (double)u * (double)u;
                 }
-                tile[ii][tx] = u;
+                tile_t[jj][ii] = u;
             }
-            __syncthreads();
-            // write X[j][i] = U[i][j]: consecutive threads take consecutive i
-#pragma unroll 4
-            for (int jj = ty; jj < EW_TILE; jj += 4) {
-                const int j = j0 + jj, i = i0 + tx;
-                if (j < sg.cols && i < sg.rows) {
-                    const float u = tile[tx][jj];
-                    store_x0(sg, (size_t)j * sg.ldn + i, u, bf16_operand);
+        }
+        __syncthreads();
+        // X0[j0 + jj][i0 + 8ig .. +7] = U[i0 + 8ig ..][j0 + jj]: thread (ig, jr) takes rows
+        // jj = jr + 32s of X, s = 0..3; 8 lanes cover 64 contiguous elements of one row
+        const int ig = threadIdx.x & 7, jr = threadIdx.x >> 3;
+        const int ix = i0 + 8 * ig;
+#pragma unroll
+        for (int sidx = 0; sidx < MT_COLS / 32; ++sidx) {
+            const int jj = jr + 32 * sidx, jx = j0 + jj;
+            if (jx >= sg.cols || ix >= sg.rows) continue;
+            float u[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) u[q] = tile_t[jj][8 * ig + q];
+            const size_t xo = (size_t)jx * sg.ldn + ix;
+            if (ix + 7 < sg.rows) {
+                if (bf16_operand) {
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) split_bf16x2(u[2 * q], u[2 * q + 1], hw[q], lw[q]);
+                    *reinterpret_cast<uint4*>(sg.xhi0 + xo) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+                    *reinterpret_cast<uint4*>(sg.xlo0 + xo) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+                } else {
+                    float4* xp = reinterpret_cast<float4*>(sg.xf0 + xo);
+                    xp[0] = make_float4(u[0], u[1], u[2], u[3]);
+                    xp[1] = make_float4(u[4], u[5], u[6], u[7]);
                 }
+            } else {
+#pragma unroll
+                for (int q = 0; q < 8; ++q)
+                    if (ix + q < sg.rows) store_x0(sg, xo + q, u[q], bf16_operand);
             }
         }
     }

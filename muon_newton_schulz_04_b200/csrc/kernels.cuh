@@ -175,6 +175,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 constexpr int EW_THREADS = 256;
 constexpr int EW_FLAT_ELEMS = 8192;      // elements per block on the flat path
-constexpr int EW_TILE = 64;              // transpose tile edge
+constexpr int EW_TILE = 64;              // transpose tile edge of the apply kernel
+constexpr int MT_ROWS = 64, MT_COLS = 128;   // transpose tile of the momentum kernel (rows x cols of W)
 
 }  // namespace muon
