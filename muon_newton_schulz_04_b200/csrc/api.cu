@@ -102,8 +102,9 @@ struct muon_handle {
     std::vector<Pending> pending;
     double t_ms[MUON_TIMING_KINDS] = {};
     int t_n[MUON_TIMING_KINDS] = {};
-    // muon_step_host: side stream for copies that overlap the GEMMs, and its events
-    cudaStream_t side = nullptr;
+    // muon_step_host: side streams for copies that overlap the GEMMs (W up, B down),
+    // and their events
+    cudaStream_t side = nullptr, side2 = nullptr;
     // captured launch sequence of muon_step / muon_orthogonalize (replayed while the
     // plan, the caller's pointers and the configuration stay the same)
     bool graphs = true;
@@ -345,7 +346,7 @@ muon_status encode_map(muon_handle* h, CUtensorMap* m, const void* base, int col
 // columns, one 64-byte row), with the 64-byte swizzle whose span is one box row.
 muon_status encode_epi_map(muon_handle* h, CUtensorMap* m, const void* base, int cols, int rows, int count, int ld) {
     return encode_map_box(h, m, base, cols, rows, count, ld, tc_gemm_epi_cols(), tc_gemm_epi_rows(),
-                          CU_TENSOR_MAP_SWIZZLE_64B);
+                          tc_gemm_epi_cols() == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
 bool is_bf16_path(const muon_handle* h) { return h->cfg.precision == MUON_PREC_BF16; }
@@ -866,15 +867,17 @@ muon_status muon_step_host(muon_handle* h, const muon_group* groups, int n_group
     std::vector<muon_group> dg_groups(groups, groups + n_groups);
     if (!h->side) {
         CUDA_TRY(h, cudaStreamCreateWithFlags(&h->side, cudaStreamNonBlocking));
+        CUDA_TRY(h, cudaStreamCreateWithFlags(&h->side2, cudaStreamNonBlocking));
         cudaEvent_t* evs[4] = {&h->ev_start, &h->ev_w, &h->ev_k1, &h->ev_done};
         for (cudaEvent_t* e : evs) CUDA_TRY(h, cudaEventCreateWithFlags(e, cudaEventDisableTiming));
     }
-    // The side stream starts after everything already queued on s (the staging
-    // area may still be in use by the previous call).  G and B go up on s; W goes
-    // up on the side stream and is waited for only before the weight update; B comes
-    // back on the side stream as soon as the momentum kernel has finished with it.
-    CUDA_TRY(h, cudaEventRecord(h->ev_start, s));
-    CUDA_TRY(h, cudaStreamWaitEvent(h->side, h->ev_start, 0));
+    // G and B go up first, on s, with the whole host-to-device bandwidth: the momentum
+    // kernel needs them.  W goes up afterwards on one side stream, while the
+    // Newton-Schulz GEMMs run, and is waited for only before the weight update; B comes
+    // back on a second side stream as soon as the momentum kernel has finished with it,
+    // in the other direction of the link, so that it overlaps W's upload.  Both side
+    // streams start after everything already queued on s (the staging area may still be
+    // in use by the previous call).
     int mi = 0;
     for (int i = 0; i < n_groups; ++i) {
         const size_t e = (size_t)groups[i].rows * groups[i].cols;
@@ -885,23 +888,31 @@ muon_status muon_step_host(muon_handle* h, const muon_group* groups, int n_group
             void* g = base + og[mi];
             CUDA_TRY(h, cudaMemcpyAsync(g, groups[i].G[k], gsz, cudaMemcpyHostToDevice, s));
             CUDA_TRY(h, cudaMemcpyAsync(b, groups[i].B[k], e * 4, cudaMemcpyHostToDevice, s));
-            CUDA_TRY(h, cudaMemcpyAsync(w, groups[i].W[k], e * 4, cudaMemcpyHostToDevice, h->side));
             Wd[i].push_back(w); Bd[i].push_back(b); Gd[i].push_back(g);
         }
         dg_groups[i].W = Wd[i].data(); dg_groups[i].B = Bd[i].data(); dg_groups[i].G = Gd[i].data();
+    }
+    CUDA_TRY(h, cudaEventRecord(h->ev_start, s));
+    CUDA_TRY(h, cudaStreamWaitEvent(h->side, h->ev_start, 0));
+    mi = 0;
+    for (int i = 0; i < n_groups; ++i) {
+        const size_t e = (size_t)groups[i].rows * groups[i].cols;
+        for (int k = 0; k < groups[i].count; ++k, ++mi)
+            CUDA_TRY(h, cudaMemcpyAsync(base + ow[mi], groups[i].W[k], e * 4, cudaMemcpyHostToDevice, h->side));
     }
     CUDA_TRY(h, cudaEventRecord(h->ev_w, h->side));
     Hooks hooks;
     hooks.w_ready = h->ev_w;
     hooks.after_momentum = [&]() -> muon_status {
         CUDA_TRY(h, cudaEventRecord(h->ev_k1, s));
-        CUDA_TRY(h, cudaStreamWaitEvent(h->side, h->ev_k1, 0));
+        CUDA_TRY(h, cudaStreamWaitEvent(h->side2, h->ev_k1, 0));
         int j = 0;
         for (int i = 0; i < n_groups; ++i) {
             const size_t e = (size_t)groups[i].rows * groups[i].cols;
             for (int k = 0; k < groups[i].count; ++k, ++j)
-                CUDA_TRY(h, cudaMemcpyAsync(groups[i].B[k], base + ob[j], e * 4, cudaMemcpyDeviceToHost, h->side));
+                CUDA_TRY(h, cudaMemcpyAsync(groups[i].B[k], base + ob[j], e * 4, cudaMemcpyDeviceToHost, h->side2));
         }
+        CUDA_TRY(h, cudaEventRecord(h->ev_done, h->side2));
         return MUON_OK;
     };
     if ((st = step_device(h, dg_groups.data(), n_groups, s, &hooks)) != MUON_OK) return st;
@@ -911,7 +922,6 @@ muon_status muon_step_host(muon_handle* h, const muon_group* groups, int n_group
         for (int k = 0; k < groups[i].count; ++k, ++mi)
             CUDA_TRY(h, cudaMemcpyAsync(groups[i].W[k], base + ow[mi], e * 4, cudaMemcpyDeviceToHost, s));
     }
-    CUDA_TRY(h, cudaEventRecord(h->ev_done, h->side));
     CUDA_TRY(h, cudaStreamWaitEvent(s, h->ev_done, 0));
     return MUON_OK;
 }
@@ -1308,6 +1318,7 @@ muon_status muon_destroy(muon_handle* h) {
         cudaEvent_t evs[4] = {h->ev_start, h->ev_w, h->ev_k1, h->ev_done};
         for (cudaEvent_t e : evs) if (e) cudaEventDestroy(e);
         if (h->side) cudaStreamDestroy(h->side);
+        if (h->side2) cudaStreamDestroy(h->side2);
         if (h->gexec) cudaGraphExecDestroy(h->gexec);
         if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
         if (h->ws.ptr) cudaFree(h->ws.ptr);

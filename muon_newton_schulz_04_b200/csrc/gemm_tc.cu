@@ -77,7 +77,11 @@ constexpr int S2_B = 128 * BK * 2;            // 16 KiB: this CTA's 128 columns 
 #ifndef MUON_S2U_STAGES
 #define MUON_S2U_STAGES 4
 #endif
-constexpr int EU_COLS = 32;                         // columns per chunk: one 64-byte bf16 box row
+#ifndef MUON_EU_COLS
+#define MUON_EU_COLS 32
+#endif
+constexpr int EU_COLS = MUON_EU_COLS;               // columns per chunk: one 64- or 128-byte bf16 box row
+static_assert(EU_COLS == 32 || EU_COLS == 64, "epilogue chunks are 32 or 64 columns");
 constexpr int EU_ROWS = 128;                        // rows per chunk: the CTA's accumulator rows
 constexpr int EU_DEPTH = MUON_EU_DEPTH;
 constexpr int EU_ROW_BYTES = EU_COLS * 2;
@@ -635,11 +639,13 @@ __device__ __forceinline__ EuChunk eu_chunk(int4 tile, int4 sk, int gm, int gn, 
     return ch;
 }
 
-// Byte offset of 16-byte slot k of row r inside a box with 64-byte rows and the
-// 64-byte swizzle (slot ^= (r >> 1) & 3): the 8 lanes of a quarter-warp access read
-// 8 distinct slots of a 128-byte span, so the row-per-lane accesses are conflict free.
+// Byte offset of 16-byte slot k of row r inside a box with EU_ROW_BYTES-byte rows and
+// the swizzle of that span (64B: slot ^= (r >> 1) & 3; 128B: slot ^= r & 7): the 8
+// lanes of a quarter-warp access read 8 distinct 16-byte bank groups, so the
+// row-per-lane accesses are conflict free.
 __device__ __forceinline__ uint32_t eu_off(int r, int k) {
-    return (uint32_t)(r * EU_ROW_BYTES + ((k ^ ((r >> 1) & 3)) << 4));
+    if (EU_ROW_BYTES == 64) return (uint32_t)(r * EU_ROW_BYTES + ((k ^ ((r >> 1) & 3)) << 4));
+    return (uint32_t)(r * EU_ROW_BYTES + ((k ^ (r & 7)) << 4));
 }
 
 // X' = alpha * acc + beta * (hi + lo) for this lane's row of one chunk, in place in
@@ -647,10 +653,10 @@ __device__ __forceinline__ uint32_t eu_off(int r, int k) {
 // values of the stored pair, hi' + lo' (fp32 bits), for the weight update.
 template <bool APPLY>
 __device__ __forceinline__ void eu_compute(uint32_t hi_s, uint32_t lo_s, int lane, float alpha, float beta,
-                                           uint32_t (&v)[EU_COLS]) {
+                                           uint32_t (&v)[32], int kbase = 0) {
 #pragma unroll
-    for (int k = 0; k < EU_COLS / 8; ++k) {
-        const uint32_t off = eu_off(lane, k);
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t off = eu_off(lane, kbase + k);
         const uint4 hv = lds128(hi_s + off), lv = lds128(lo_s + off);
         const uint32_t h4[4] = {hv.x, hv.y, hv.z, hv.w};
         const uint32_t l4[4] = {lv.x, lv.y, lv.z, lv.w};
@@ -971,44 +977,54 @@ __device__ __forceinline__ bool update_epilogue_compute(const GemmParams& p, uin
             const EuChunk ch = eu_chunk(tile, sk, gm, gn, c, (int)rank, half);
             if (kind == 2) {
                 // a later K range of a split tile: its raw partial sum goes to the slot
-                uint32_t v[EU_COLS];
-                tmem_ld_32x32b_x32(tacc + (uint32_t)ch.tcol, v);
-                tmem_ld_wait();
-                float4* dst = reinterpret_cast<float4*>(sk_row + ch.tcol);
+                for (int sub = 0; sub < EU_COLS / 32; ++sub) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(tacc + (uint32_t)(ch.tcol + 32 * sub), v);
+                    tmem_ld_wait();
+                    float4* dst = reinterpret_cast<float4*>(sk_row + ch.tcol + 32 * sub);
 #pragma unroll
-                for (int qq = 0; qq < EU_COLS / 4; ++qq)
-                    dst[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
-                                          __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
+                    for (int qq = 0; qq < 8; ++qq)
+                        dst[qq] = make_float4(__uint_as_float(v[4 * qq]), __uint_as_float(v[4 * qq + 1]),
+                                              __uint_as_float(v[4 * qq + 2]), __uint_as_float(v[4 * qq + 3]));
+                }
                 continue;
             }
             if (!ch.load) continue;               // the CTA's rows or the columns lie outside the matrix
-            uint32_t v[EU_COLS];
-            tmem_ld_32x32b_x32(tacc + (uint32_t)ch.tcol, v);
-            tmem_ld_wait();
-            if (kind == 1) {
-                for (int sl = 0; sl < nsl; ++sl) {
-                    const float4* src = reinterpret_cast<const float4*>(sk_row + (size_t)sl * SK_SLOT_FLOATS + ch.tcol);
-#pragma unroll
-                    for (int qq = 0; qq < EU_COLS / 4; ++qq) {
-                        const float4 x = __ldcg(src + qq);
-                        v[4 * qq + 0] = __float_as_uint(__uint_as_float(v[4 * qq + 0]) + x.x);
-                        v[4 * qq + 1] = __float_as_uint(__uint_as_float(v[4 * qq + 1]) + x.y);
-                        v[4 * qq + 2] = __float_as_uint(__uint_as_float(v[4 * qq + 2]) + x.z);
-                        v[4 * qq + 3] = __float_as_uint(__uint_as_float(v[4 * qq + 3]) + x.w);
-                    }
-                }
-            }
             const uint32_t b = consumed % EU_DEPTH;
             ok = mbar_wait(&efull[b], (consumed / EU_DEPTH) & 1u, abort_flag, p.err, ERR_EPILOGUE);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             const uint32_t hi_s = smem_u32(ebuf + b * EU_BUF) + (uint32_t)(q * 32 * EU_ROW_BYTES), lo_s = hi_s + EU_BOX;
-            if (sg != nullptr) eu_compute<true>(hi_s, lo_s, (int)lane, alpha, beta, v);
-            else eu_compute<false>(hi_s, lo_s, (int)lane, alpha, beta, v);
+            // 32 accumulator columns at a time (one tcgen05.ld)
+#pragma unroll 1
+            for (int sub = 0; sub < EU_COLS / 32; ++sub) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(tacc + (uint32_t)(ch.tcol + 32 * sub), v);
+                tmem_ld_wait();
+                if (kind == 1) {
+                    for (int sl = 0; sl < nsl; ++sl) {
+                        const float4* src =
+                            reinterpret_cast<const float4*>(sk_row + (size_t)sl * SK_SLOT_FLOATS + ch.tcol + 32 * sub);
+#pragma unroll
+                        for (int qq = 0; qq < 8; ++qq) {
+                            const float4 x = __ldcg(src + qq);
+                            v[4 * qq + 0] = __float_as_uint(__uint_as_float(v[4 * qq + 0]) + x.x);
+                            v[4 * qq + 1] = __float_as_uint(__uint_as_float(v[4 * qq + 1]) + x.y);
+                            v[4 * qq + 2] = __float_as_uint(__uint_as_float(v[4 * qq + 2]) + x.z);
+                            v[4 * qq + 3] = __float_as_uint(__uint_as_float(v[4 * qq + 3]) + x.w);
+                        }
+                    }
+                }
+                if (sg != nullptr) {
+                    eu_compute<true>(hi_s, lo_s, (int)lane, alpha, beta, v, 4 * sub);
+                    if (row < gm) apply_row<32>(p, gi, *sg, row, ch.col0 + 32 * sub, v);
+                } else {
+                    eu_compute<false>(hi_s, lo_s, (int)lane, alpha, beta, v, 4 * sub);
+                }
+            }
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(&edone[b]);
             ++consumed;
-            if (sg != nullptr && row < gm) apply_row<EU_COLS>(p, gi, *sg, row, ch.col0, v);
         }
         if (!ok) break;
         tc_fence_before();
