@@ -54,6 +54,7 @@ struct Plan {
     std::vector<EwSeg> segs;             // shape part filled at plan time
     // tile lists (tensor-core path)
     int n_gram = 0, n_poly = 0, n_upd = 0;
+    int var[3] = {1, 0, 0};              // two-CTA shared-memory configuration per phase
     // device addresses inside the workspace
     int4* d_tiles_gram = nullptr; int4* d_tiles_poly = nullptr; int4* d_tiles_upd = nullptr;
     // two-CTA kernel: per-phase unit lists (plan.h) and the split-tile partial sums
@@ -349,6 +350,16 @@ muon_status encode_epi_map(muon_handle* h, CUtensorMap* m, const void* base, int
                           tc_gemm_epi_cols() == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+// The two boxes of a symmetric m x m output (A or P) for the Gram / polynomial
+// epilogue: [0] the direct box (as encode_epi_map), [1] its transpose, tc_gemm_epi_cols()
+// rows of tc_gemm_epi_rows() columns, unswizzled, for the mirrored stores.
+muon_status encode_sym_maps(muon_handle* h, CUtensorMap* m2, const void* base, int mdim, int count, int ld) {
+    muon_status st = encode_epi_map(h, &m2[0], base, mdim, mdim, count, ld);
+    if (st != MUON_OK) return st;
+    return encode_map_box(h, &m2[1], base, mdim, mdim, count, ld, tc_gemm_epi_rows(), tc_gemm_epi_cols(),
+                          CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 bool is_bf16_path(const muon_handle* h) { return h->cfg.precision == MUON_PREC_BF16; }
 
 // Persistent grid: one CTA (or one two-CTA cluster) per tile, at most one per SM.
@@ -435,6 +446,17 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
                 sk_slots = std::max(sk_slots, upl[ph].nslots);
             }
             P.unit_clusters = h->max_clusters;
+        }
+        // per phase, the shared-memory configuration for the tiles' average K
+        {
+            const std::vector<Tile>* lists[3] = {&tg, &tp, &tu};
+            const int modes[3] = {MODE_GRAM, MODE_POLY, MODE_UPDATE};
+            for (int ph = 0; ph < 3; ++ph) {
+                long long ksum = 0;
+                for (const Tile& t : *lists[ph]) ksum += ph == 0 ? P.dims[t.group].n : P.dims[t.group].m;
+                const int avg = lists[ph]->empty() ? 0 : (int)(ksum / (long long)lists[ph]->size());
+                P.var[ph] = tc_gemm_var(modes[ph], avg);
+            }
         }
         // nothing is launched with a plan that does not cover its outputs exactly once
         const std::vector<Tile>* lists[3] = {&tg, &tp, &tu};
@@ -524,6 +546,8 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
                 if ((st = encode_epi_map(h, &maps[g].xe_hi[b], base + o.xb[b], d.n, d.m, d.count, d.ldn)) != MUON_OK) return st;
             if ((st = encode_epi_map(h, &maps[g].xe_lo_in, base + o.xl, d.n, d.m, d.count, d.ldn)) != MUON_OK) return st;
             maps[g].xe_lo_out = maps[g].xe_lo_in;
+            if ((st = encode_sym_maps(h, maps[g].se_a, base + o.a, d.m, d.count, d.ldm)) != MUON_OK) return st;
+            if ((st = encode_sym_maps(h, maps[g].se_p, base + o.p, d.m, d.count, d.ldm)) != MUON_OK) return st;
             GemmGroupInfo& q = gi[g];
             q.m = d.m; q.n = d.n; q.ldm = d.ldm; q.ldn = d.ldn; q.count = d.count; q.mat_base = P.mat_base[g];
             q.xb[0] = reinterpret_cast<__nv_bfloat16*>(base + o.xb[0]);
@@ -634,10 +658,10 @@ muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStrea
             gp.tiles = P.d_tiles_gram; gp.ntiles = P.n_gram; gp.alpha = 1.f; gp.beta = 0.f;
             gp.units = P.d_units[0]; gp.unit_begin = P.d_unit_begin[0]; gp.epoch = ++h->epoch;
             gp.scale = it == 0 ? P.d_scale : nullptr;
-            TIMED(h, 2, s, launch_tc_gemm(MODE_GRAM, h->pair, gp, gemm_grid(h, P.n_gram), s));
+            TIMED(h, 2, s, launch_tc_gemm(MODE_GRAM, h->pair, gp, gemm_grid(h, P.n_gram), s, P.var[0]));
             gp.tiles = P.d_tiles_poly; gp.ntiles = P.n_poly; gp.alpha = c.ns_c; gp.beta = c.ns_b; gp.scale = nullptr;
             gp.units = P.d_units[1]; gp.unit_begin = P.d_unit_begin[1]; gp.epoch = ++h->epoch;
-            TIMED(h, 3, s, launch_tc_gemm(MODE_POLY, h->pair, gp, gemm_grid(h, P.n_poly), s));
+            TIMED(h, 3, s, launch_tc_gemm(MODE_POLY, h->pair, gp, gemm_grid(h, P.n_poly), s, P.var[1]));
             gp.tiles = P.d_tiles_upd; gp.ntiles = P.n_upd; gp.alpha = 1.f; gp.beta = c.ns_a;
             gp.units = P.d_units[2]; gp.unit_begin = P.d_unit_begin[2]; gp.epoch = ++h->epoch;
             gp.scale = it == 0 ? P.d_scale : nullptr;
@@ -649,7 +673,7 @@ muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStrea
                 gp.lr = c.lr;
                 gp.segs = P.d_segs;
             }
-            TIMED(h, 4, s, launch_tc_gemm(MODE_UPDATE, h->pair, gp, gemm_grid(h, P.n_upd), s));
+            TIMED(h, 4, s, launch_tc_gemm(MODE_UPDATE, h->pair, gp, gemm_grid(h, P.n_upd), s, P.var[2]));
         } else {
             for (size_t g = 0; g < P.dims.size(); ++g) {
                 const GroupDims& d = P.dims[g];
@@ -1138,9 +1162,12 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     gi.m = m; gi.n = n; gi.ldm = m; gi.ldn = n; gi.count = cnt; gi.mat_base = 0;
     if (phase == MUON_NS_GRAM) {
         if ((st = encode_map(h, &maps.xb_k[0], a->x_op, n, m, cnt, n, 128)) != MUON_OK) return st;
+        if ((st = encode_sym_maps(h, maps.se_a, a->out, m, cnt, m)) != MUON_OK) return st;
         gi.a = (__nv_bfloat16*)a->out;
     } else if (phase == MUON_NS_POLY) {
         if ((st = encode_map(h, &maps.a, a->a_in, m, m, cnt, m, 128)) != MUON_OK) return st;
+        if ((st = encode_sym_maps(h, maps.se_a, a->a_in, m, cnt, m)) != MUON_OK) return st;
+        if ((st = encode_sym_maps(h, maps.se_p, a->out, m, cnt, m)) != MUON_OK) return st;
         gi.a = (__nv_bfloat16*)a->a_in;
         gi.p = (__nv_bfloat16*)a->out;
     } else {
@@ -1208,7 +1235,8 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     gp.write_op = (phase == MUON_NS_UPDATE && a->out_op) ? 1 : 0;
     gp.err = h->d_err;
     const int mode = phase == MUON_NS_GRAM ? MODE_GRAM : phase == MUON_NS_POLY ? MODE_POLY : MODE_UPDATE;
-    CUDA_TRY(h, launch_tc_gemm(mode, h->pair, gp, gemm_grid(h, gp.ntiles), s));
+    CUDA_TRY(h, launch_tc_gemm(mode, h->pair, gp, gemm_grid(h, gp.ntiles), s,
+                               tc_gemm_var(mode, phase == MUON_NS_GRAM ? n : m)));
     return MUON_OK;
 }
 

@@ -57,10 +57,7 @@ constexpr int S1_B = S1_BN * BK * 2;          // 32 KiB
 constexpr int S1_SMEM = 1024 + S1_STAGES * (S1_A + S1_B) + 256 + STAGE_BYTES;
 
 // two-CTA kernel (per CTA)
-#ifndef MUON_S2_STAGES
-#define MUON_S2_STAGES 6
-#endif
-constexpr int S2_BM = 256, S2_BN = 256, S2_STAGES = MUON_S2_STAGES;
+constexpr int S2_BM = 256, S2_BN = 256;
 constexpr int S2_A = 128 * BK * 2;            // 16 KiB: this CTA's 128 rows of A
 constexpr int S2_B = 128 * BK * 2;            // 16 KiB: this CTA's 128 columns of B
 
@@ -77,39 +74,57 @@ constexpr int S2_B = 128 * BK * 2;            // 16 KiB: this CTA's 128 columns 
 #ifndef MUON_S2U_STAGES
 #define MUON_S2U_STAGES 4
 #endif
+// Gram: the epilogue loads nothing, so a ring of two boxes suffices and the operand
+// ring gets a fifth stage for its long K (n); the polynomial (K = m, A loaded for the
+// b*A term) keeps the update's ring and stages.
+#ifndef MUON_ES_DEPTH
+#define MUON_ES_DEPTH 2
+#endif
+#ifndef MUON_S2S_STAGES
+#define MUON_S2S_STAGES 5
+#endif
 #ifndef MUON_EU_COLS
 #define MUON_EU_COLS 32
 #endif
 constexpr int EU_COLS = MUON_EU_COLS;               // columns per chunk: one 64- or 128-byte bf16 box row
 static_assert(EU_COLS == 32 || EU_COLS == 64, "epilogue chunks are 32 or 64 columns");
 constexpr int EU_ROWS = 128;                        // rows per chunk: the CTA's accumulator rows
-constexpr int EU_DEPTH = MUON_EU_DEPTH;
+constexpr int EU_DEPTH = MUON_EU_DEPTH;            // update epilogue ring depth
+constexpr int ES_DEPTH = MUON_ES_DEPTH;            // ring depth of the long-K configuration
+// Two shared-memory configurations of the two-CTA kernel: VAR 0 (ring depth EU_DEPTH,
+// S2U_STAGES operand stages) for short K, VAR 1 (ES_DEPTH, S2S_STAGES) for long K.
+// The Gram always takes VAR 1 (its epilogue loads nothing); the polynomial and the
+// update choose per launch from the plan's K (launch_tc_gemm's `var`).
+__host__ __device__ constexpr int eu_depth(int var) { return var ? ES_DEPTH : EU_DEPTH; }
 constexpr int EU_ROW_BYTES = EU_COLS * 2;
 constexpr int EU_BOX = EU_ROWS * EU_ROW_BYTES;      // 8 KiB
 constexpr int EU_BUF = 2 * EU_BOX;                  // hi + lo
 constexpr int S2U_STAGES = MUON_S2U_STAGES;
+constexpr int S2S_STAGES = MUON_S2S_STAGES;
 constexpr int NUM_THREADS_U = NUM_THREADS + 64;     // + the two epilogue TMA warps
-static_assert(EU_DEPTH >= 2 && EU_DEPTH <= 6, "epilogue ring depth out of range");
+static_assert(EU_DEPTH >= 2 && EU_DEPTH <= 6 && ES_DEPTH >= 2 && ES_DEPTH <= 6, "epilogue ring depth out of range");
 
-constexpr int s2_stages(int mode) { return mode == MODE_UPDATE ? S2U_STAGES : S2_STAGES; }
-constexpr int s2_epi_bytes(int mode) { return mode == MODE_UPDATE ? 2 * EU_DEPTH * EU_BUF : STAGE_BYTES; }
-constexpr int s2_threads(int mode) { return mode == MODE_UPDATE ? NUM_THREADS_U : NUM_THREADS; }
+// Every mode of the two-CTA kernel uses the TMA epilogue (the Gram and polynomial
+// products store their symmetric output through the same ring of boxes).
+constexpr int s2_stages(int var) { return var ? S2S_STAGES : S2U_STAGES; }
+constexpr int s2_epi_bytes(int var) { return 2 * eu_depth(var) * EU_BUF; }
+constexpr int s2_threads(int) { return NUM_THREADS_U; }
 // barriers: full / empty per stage, two tfull / tempty, drain, the epilogue ring's
 // (UPDATE), then the TMEM address and the abort flag
-constexpr int s2_bar_bytes(int mode) {
-    // (+ UPDATE: the epilogue TMA warps' chunk coordinates, 2 x EU_DEPTH int4)
-    return (8 * (2 * s2_stages(mode) + 5 + (mode == MODE_UPDATE ? 4 * EU_DEPTH : 0)) + 8 + 16 +
-            (mode == MODE_UPDATE ? 2 * EU_DEPTH * 16 : 0) + 127) / 128 * 128;
+constexpr int s2_bar_bytes(int var) {
+    // (+ the epilogue TMA warps' chunk coordinates, 2 x ring depth int4)
+    return (8 * (2 * s2_stages(var) + 5 + 4 * eu_depth(var)) + 8 + 16 + 2 * eu_depth(var) * 16 + 127) / 128 * 128;
 }
 // [operand ring][epilogue buffers][barriers]; the ring and the buffers are 1024-byte aligned
-constexpr int s2_smem(int mode) {
-    return 1024 + s2_stages(mode) * (S2_A + S2_B) + s2_epi_bytes(mode) + s2_bar_bytes(mode);
+constexpr int s2_smem(int var) {
+    return 1024 + s2_stages(var) * (S2_A + S2_B) + s2_epi_bytes(var) + s2_bar_bytes(var);
 }
-constexpr int S2_SMEM = s2_smem(MODE_GRAM);
-constexpr int S2U_SMEM = s2_smem(MODE_UPDATE);
+constexpr int S2_SMEM = s2_smem(1);
+constexpr int S2U_SMEM = s2_smem(0);
 static_assert(S1_SMEM <= 232448 && S2_SMEM <= 232448 && S2U_SMEM <= 232448,
               "dynamic shared memory above the 227 KiB limit");
-static_assert((s2_stages(MODE_UPDATE) * (S2_A + S2_B)) % 1024 == 0 && EU_BUF % 1024 == 0, "buffer alignment");
+static_assert((s2_stages(0) * (S2_A + S2_B)) % 1024 == 0 && (s2_stages(1) * (S2_A + S2_B)) % 1024 == 0 &&
+              EU_BUF % 1024 == 0, "buffer alignment");
 
 // error codes written to the device error word when a bounded wait gives up
 constexpr int ERR_PRODUCER = 0x101, ERR_MMA_SLOT = 0x102, ERR_MMA_ACC = 0x103, ERR_EPILOGUE = 0x104,
@@ -865,14 +880,55 @@ __device__ __forceinline__ void prefetch_w_row(const GemmParams& p, const GemmGr
     }
 }
 
-// The TMA warp of one column half of the two-CTA UPDATE epilogue (one elected
+// GRAM / POLY epilogue of this lane's row (brow, 0..127 in the chunk's boxes) of one
+// chunk: y = alpha * acc (+ beta * A for the polynomial, read from the D box) written
+// as bf16 to the D box in place (64-byte swizzle) and, for a tile off the diagonal,
+// to the transposed box T[c][brow] (32 rows of 128 columns, no swizzle), whose store
+// writes the mirrored elements.  d_s: the D box row of the warp's first row.
+template <int MODE>
+__device__ __forceinline__ void sym_compute(uint32_t d_s, uint32_t t_s, int lane, int brow, float alpha, float beta,
+                                            const uint32_t (&v)[32], bool offdiag, int kbase = 0) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const uint32_t off = eu_off(lane, kbase + k);
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = alpha * __uint_as_float(v[8 * k + e]);
+        if (MODE == MODE_POLY) {
+            const uint4 av = lds128(d_s + off);
+            const uint32_t a4[4] = {av.x, av.y, av.z, av.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                y[2 * e] += beta * bf16_bits_lo(a4[e]);
+                y[2 * e + 1] += beta * bf16_bits_hi(a4[e]);
+            }
+        }
+        const uint32_t w0 = pack_bf16x2(y[0], y[1]), w1 = pack_bf16x2(y[2], y[3]);
+        const uint32_t w2 = pack_bf16x2(y[4], y[5]), w3 = pack_bf16x2(y[6], y[7]);
+        sts128(d_s + off, make_uint4(w0, w1, w2, w3));
+        if (offdiag) {
+            const uint32_t w[4] = {w0, w1, w2, w3};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t c = (uint32_t)(8 * (kbase + k) + 2 * e);
+                asm volatile("st.shared.b16 [%0], %1;" :: "r"(t_s + c * 256u + (uint32_t)brow * 2u),
+                             "h"((unsigned short)(w[e] & 0xFFFFu)) : "memory");
+                asm volatile("st.shared.b16 [%0], %1;" :: "r"(t_s + (c + 1u) * 256u + (uint32_t)brow * 2u),
+                             "h"((unsigned short)(w[e] >> 16)) : "memory");
+            }
+        }
+    }
+}
+
+// The TMA warp of one column half of the two-CTA epilogue (one elected
 // thread): walks the half's load chunks of every unit of its cluster in order,
 // loading chunk j + EU_DEPTH - 1 into the ring once chunk j - 1's stores have read
 // their buffer, and storing chunk j once the half's four compute warps have arrived
 // on its done barrier.  Returns false when a bounded wait gave up.
-__device__ __forceinline__ bool update_epilogue_tma(const GemmParams& p, uint32_t rank, int half, uint8_t* ebuf,
-                                                    uint64_t* efull, uint64_t* edone, int4* coord,
-                                                    volatile int* abort_flag, int cid) {
+template <int MODE, int D>
+__device__ __forceinline__ bool pair_epilogue_tma(const GemmParams& p, uint32_t rank, int half, uint8_t* ebuf,
+                                                  uint64_t* efull, uint64_t* edone, int4* coord,
+                                                  volatile int* abort_flag, int cid) {
     const int u_begin = p.unit_begin[cid], u_end = p.unit_begin[cid + 1];
     // next (unit, chunk) to look at, with that unit's descriptor and group shape
     int iu = u_begin - 1, ic = 0, inch = 0, igm = 0, ign = 0;
@@ -881,38 +937,52 @@ __device__ __forceinline__ bool update_epilogue_tma(const GemmParams& p, uint32_
     uint32_t issued = 0, stored = 0;
     bool more = true, ok = true;
     while (true) {
-        // load chunk i once the stores of chunk i - EU_DEPTH have read its buffer: after
+        // load chunk i once the stores of chunk i - D have read its buffer: after
         // the wait below, every store but the last one has
-        while (more && issued + 1 < stored + EU_DEPTH) {
+        while (more && issued + 1 < stored + D) {
             if (ic >= inch) {
                 if (++iu >= u_end) { more = false; break; }
                 itile = p.units[2 * iu];
                 isk = p.units[2 * iu + 1];
                 inch = eu_nchunks(isk);
                 igm = p.groups[itile.x].m;
-                ign = p.groups[itile.x].n;
+                ign = MODE == MODE_UPDATE ? p.groups[itile.x].n : igm;     // GRAM / POLY: m x m output
                 ic = 0;
                 continue;
             }
             const EuChunk ch = eu_chunk(itile, isk, igm, ign, ic, (int)rank, half);
             ++ic;
             if (!ch.load) continue;
-            const uint32_t b = issued % EU_DEPTH;
+            const uint32_t b = issued % D;
             uint8_t* dst = ebuf + b * EU_BUF;
             const GemmMaps& mp = p.maps[ch.g];
             coord[b] = make_int4(ch.g, ch.mat, ch.row0, ch.col0);
-            mbar_arrive_expect_tx(&efull[b], EU_BUF);
-            tma_load_3d(dst, &mp.xe_hi[p.parity], &efull[b], ch.col0, ch.row0, ch.mat);
-            tma_load_3d(dst + EU_BOX, &mp.xe_lo_in, &efull[b], ch.col0, ch.row0, ch.mat);
+            if (MODE == MODE_UPDATE) {
+                mbar_arrive_expect_tx(&efull[b], EU_BUF);
+                tma_load_3d(dst, &mp.xe_hi[p.parity], &efull[b], ch.col0, ch.row0, ch.mat);
+                tma_load_3d(dst + EU_BOX, &mp.xe_lo_in, &efull[b], ch.col0, ch.row0, ch.mat);
+            } else if (MODE == MODE_POLY) {
+                mbar_arrive_expect_tx(&efull[b], EU_BOX);     // A, for the b*A term
+                tma_load_3d(dst, &mp.se_a[0], &efull[b], ch.col0, ch.row0, ch.mat);
+            } else {
+                mbar_arrive(&efull[b]);                        // GRAM: the buffer is free
+            }
             ++issued;
         }
         if (stored == issued) break;
-        const uint32_t b = stored % EU_DEPTH;
-        if (!mbar_wait(&edone[b], (stored / EU_DEPTH) & 1u, abort_flag, p.err, ERR_EPILOGUE)) { ok = false; break; }
+        const uint32_t b = stored % D;
+        if (!mbar_wait(&edone[b], (stored / D) & 1u, abort_flag, p.err, ERR_EPILOGUE)) { ok = false; break; }
         const int4 cd = coord[b];
         const GemmMaps& mp = p.maps[cd.x];
-        tma_store_3d(&mp.xe_hi[p.parity ^ 1], ebuf + b * EU_BUF, cd.w, cd.z, cd.y);
-        tma_store_3d(&mp.xe_lo_out, ebuf + b * EU_BUF + EU_BOX, cd.w, cd.z, cd.y);
+        if (MODE == MODE_UPDATE) {
+            tma_store_3d(&mp.xe_hi[p.parity ^ 1], ebuf + b * EU_BUF, cd.w, cd.z, cd.y);
+            tma_store_3d(&mp.xe_lo_out, ebuf + b * EU_BUF + EU_BOX, cd.w, cd.z, cd.y);
+        } else {
+            const CUtensorMap* out = MODE == MODE_GRAM ? mp.se_a : mp.se_p;
+            tma_store_3d(&out[0], ebuf + b * EU_BUF, cd.w, cd.z, cd.y);
+            // a tile off the diagonal also writes its mirror: rows col0.., columns row0..
+            if ((cd.z / S2_BM) != (cd.w / S2_BN)) tma_store_3d(&out[1], ebuf + b * EU_BUF + EU_BOX, cd.z, cd.w, cd.y);
+        }
         bulk_commit();
         ++stored;
         bulk_wait_read<1>();              // every store but this one has read its buffer
@@ -921,7 +991,7 @@ __device__ __forceinline__ bool update_epilogue_tma(const GemmParams& p, uint32_
     // loads still in flight (after an abort) must land before the CTA retires
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t i = stored; i < issued; ++i)
-        while (!mbar_try_wait(&efull[i % EU_DEPTH], (i / EU_DEPTH) & 1u) && globaltimer_ns() - t0 < 100000000ull) { }
+        while (!mbar_try_wait(&efull[i % D], (i / D) & 1u) && globaltimer_ns() - t0 < 100000000ull) { }
     return ok;
 }
 
@@ -931,10 +1001,11 @@ __device__ __forceinline__ bool update_epilogue_tma(const GemmParams& p, uint32_
 // layout) and rewrites its row of both boxes in place; the warp then arrives on the
 // chunk's done barrier for the TMA warp.  The fused weight update (last iteration)
 // follows from registers.  Returns false when a bounded wait gave up.
-__device__ __forceinline__ bool update_epilogue_compute(const GemmParams& p, uint32_t rank, uint32_t warp,
-                                                        uint32_t tmem_base, uint8_t* ebuf, uint64_t* efull,
-                                                        uint64_t* edone, uint64_t* tfull, uint64_t* tempty,
-                                                        volatile int* abort_flag, int cid) {
+template <int MODE, int D>
+__device__ __forceinline__ bool pair_epilogue_compute(const GemmParams& p, uint32_t rank, uint32_t warp,
+                                                      uint32_t tmem_base, uint8_t* ebuf, uint64_t* efull,
+                                                      uint64_t* edone, uint64_t* tfull, uint64_t* tempty,
+                                                      volatile int* abort_flag, int cid) {
     const uint32_t lane = threadIdx.x & 31u;
     const int q = (int)(warp & 3u), half = (int)((warp - 2) >> 2);
     const int u_begin = p.unit_begin[cid], u_end = p.unit_begin[cid + 1];
@@ -947,11 +1018,12 @@ __device__ __forceinline__ bool update_epilogue_compute(const GemmParams& p, uin
         const int4 sk = p.units[2 * u + 1];
         const int kind = sk.z & 0xFF, nh = sk.z >> 8, slot = sk.w & 0xFFFF, nsl = sk.w >> 16;
         const GemmGroupInfo& gi = p.groups[tile.x];
-        const int gm = gi.m, gn = gi.n;
+        const int gm = gi.m, gn = MODE == MODE_UPDATE ? gi.n : gi.m;
         const uint32_t acc = local & 1;
         const uint32_t acc_phase = (local >> 1) & 1;
         const int row = tile.z * S2_BM + (int)rank * 128 + brow;
-        if (kind != 2)
+        const bool offdiag = tile.z != tile.w;
+        if (MODE == MODE_UPDATE && kind != 2)
             prefetch_w_row(p, gi, tile.y, row, tile.w * S2_BN + (nh ? (nh - 1) * 128 + half * 64 : half * 128),
                            nh ? 64 : 128);
         ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, ERR_EPILOGUE);
@@ -964,14 +1036,15 @@ __device__ __forceinline__ bool update_epilogue_compute(const GemmParams& p, uin
         tc_fence_after();
         float alpha = p.alpha, beta = p.beta;
         if (p.scale != nullptr) {
+            // first iteration: A0 = s^2 U U^T, X1 = s P U + a s U
             const float sc = p.scale[gi.mat_base + tile.y];
-            alpha *= sc;
-            beta *= sc;
+            alpha *= MODE == MODE_GRAM ? sc * sc : sc;
+            if (MODE == MODE_UPDATE) beta *= sc;
         }
         float* sk_row = kind == 0 ? nullptr
                       : p.sk_partial + (size_t)slot * SK_SLOT_FLOATS + ((size_t)rank * 128 + brow) * 256;
         const uint32_t tacc = tmem_base + acc * ACC_COLS + (((uint32_t)q * 32u) << 16);
-        const EwSeg* sg = p.apply_mode != 0 ? &p.segs[gi.mat_base + tile.y] : nullptr;
+        const EwSeg* sg = (MODE == MODE_UPDATE && p.apply_mode != 0) ? &p.segs[gi.mat_base + tile.y] : nullptr;
         const int nch = (nh ? 64 : 128) / EU_COLS;
         for (int c = 0; c < nch; ++c) {
             const EuChunk ch = eu_chunk(tile, sk, gm, gn, c, (int)rank, half);
@@ -990,8 +1063,8 @@ __device__ __forceinline__ bool update_epilogue_compute(const GemmParams& p, uin
                 continue;
             }
             if (!ch.load) continue;               // the CTA's rows or the columns lie outside the matrix
-            const uint32_t b = consumed % EU_DEPTH;
-            ok = mbar_wait(&efull[b], (consumed / EU_DEPTH) & 1u, abort_flag, p.err, ERR_EPILOGUE);
+            const uint32_t b = consumed % D;
+            ok = mbar_wait(&efull[b], (consumed / D) & 1u, abort_flag, p.err, ERR_EPILOGUE);
             if (!__all_sync(0xffffffffu, ok)) { ok = false; break; }
             const uint32_t hi_s = smem_u32(ebuf + b * EU_BUF) + (uint32_t)(q * 32 * EU_ROW_BYTES), lo_s = hi_s + EU_BOX;
             // 32 accumulator columns at a time (one tcgen05.ld)
@@ -1014,7 +1087,11 @@ __device__ __forceinline__ bool update_epilogue_compute(const GemmParams& p, uin
                         }
                     }
                 }
-                if (sg != nullptr) {
+                if (MODE != MODE_UPDATE) {
+                    // hi_s: the D box rows of this warp; the T box follows the D box
+                    sym_compute<MODE>(hi_s, smem_u32(ebuf + b * EU_BUF) + EU_BOX, (int)lane, brow, alpha, beta, v,
+                                      offdiag, 4 * sub);
+                } else if (sg != nullptr) {
                     eu_compute<true>(hi_s, lo_s, (int)lane, alpha, beta, v, 4 * sub);
                     if (row < gm) apply_row<32>(p, gi, *sg, row, ch.col0 + 32 * sub, v);
                 } else {
@@ -1045,29 +1122,29 @@ __device__ __forceinline__ bool update_epilogue_compute(const GemmParams& p, uin
 
 // ============================================================================ two-CTA kernel
 
-template <int MODE>
+template <int MODE, int VAR>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(s2_threads(MODE), 1)
 ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
-    constexpr int STAGES = s2_stages(MODE);
+    constexpr int STAGES = s2_stages(VAR);
+    constexpr int ED = eu_depth(VAR);                  // epilogue ring depth
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * S2_A;
     uint8_t* sE = smem + STAGES * (S2_A + S2_B);          // epilogue buffers
-    uint64_t* full = reinterpret_cast<uint64_t*>(sE + s2_epi_bytes(MODE));
+    uint64_t* full = reinterpret_cast<uint64_t*>(sE + s2_epi_bytes(VAR));
     uint64_t* empty = full + STAGES;
     uint64_t* tfull = empty + STAGES;
     uint64_t* tempty = tfull + 2;
     uint64_t* drain = tempty + 2;
-    uint64_t* ebar = drain + 1;                            // UPDATE: EU_DEPTH per epilogue warp
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + (MODE == MODE_UPDATE ? 4 * EU_DEPTH : 0));
+    uint64_t* ebar = drain + 1;                            // UPDATE: ED per epilogue warp
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ebar + 4 * ED);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    // UPDATE: 2 x EU_DEPTH chunk coordinates after the TMEM address and the abort flag,
-    // rounded up to a 16-byte boundary
+    // 2 x ED chunk coordinates after the TMEM address and the abort flag, rounded
+    // up to a 16-byte boundary
     int4* ecoord = reinterpret_cast<int4*>((reinterpret_cast<uintptr_t>(tmem_slot + 2) + 15) & ~uintptr_t(15));
 
     const uint32_t warp = warp_id();
-    const uint32_t lane = threadIdx.x & 31u;
     const uint32_t rank = cluster_ctarank();          // 0: issues the MMA
     const int cid = (int)cluster_id_x();               // index of this pair's unit list
 
@@ -1081,11 +1158,10 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
             mbar_init(&tempty[b], 2 * NUM_EPI_WARPS); // used in CTA 0: epilogue warps of both CTAs
         }
         mbar_init(drain, 1);
-        if (MODE == MODE_UPDATE)
-            for (int h = 0; h < 2; ++h)
-                for (int i = 0; i < EU_DEPTH; ++i) {
-                    mbar_init(&ebar[h * 2 * EU_DEPTH + i], 1);                  // full: the TMA warp's expect_tx
-                    mbar_init(&ebar[h * 2 * EU_DEPTH + EU_DEPTH + i], 4);       // done: the half's compute warps
+        for (int h = 0; h < 2; ++h)
+                for (int i = 0; i < ED; ++i) {
+                    mbar_init(&ebar[h * 2 * ED + i], 1);                  // full: the TMA warp's expect_tx
+                    mbar_init(&ebar[h * 2 * ED + ED + i], 4);       // done: the half's compute warps
                 }
         *abort_flag = 0;
         fence_barrier_init();
@@ -1192,64 +1268,17 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
                 while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 100000000ull) { }
             }
         }
-    } else if (MODE == MODE_UPDATE) {
-        // ring of column half h: buffers sE + h * EU_DEPTH * EU_BUF, barriers
-        // ebar[4h * ...]: EU_DEPTH full (TMA loads), then EU_DEPTH done (compute warps)
+    } else {
+        // ring of column half h: buffers sE + h * ED * EU_BUF, barriers
+        // ebar[2h * ED ...]: ED full (TMA loads), then ED done (compute warps)
         if (warp < 2 + NUM_EPI_WARPS) {
             const int h = (int)((warp - 2) >> 2);
-            update_epilogue_compute(p, rank, warp, tmem_base, sE + h * (EU_DEPTH * EU_BUF), ebar + h * 2 * EU_DEPTH,
-                                    ebar + h * 2 * EU_DEPTH + EU_DEPTH, tfull, tempty, abort_flag, cid);
+            pair_epilogue_compute<MODE, ED>(p, rank, warp, tmem_base, sE + h * (ED * EU_BUF), ebar + h * 2 * ED,
+                                        ebar + h * 2 * ED + ED, tfull, tempty, abort_flag, cid);
         } else if (elect_one()) {
             const int h = (int)(warp - 2 - NUM_EPI_WARPS);
-            update_epilogue_tma(p, rank, h, sE + h * (EU_DEPTH * EU_BUF), ebar + h * 2 * EU_DEPTH,
-                                ebar + h * 2 * EU_DEPTH + EU_DEPTH, ecoord + h * EU_DEPTH, abort_flag, cid);
-        }
-    } else {
-        const uint32_t q = warp & 3u;
-        const uint32_t half = (warp - 2) >> 2;
-        float* stage = reinterpret_cast<float*>(sE) + (warp - 2) * STAGE_FLOATS;
-        int local = 0;
-        const int u_end = p.unit_begin[cid + 1];
-        for (int u = p.unit_begin[cid]; u < u_end; ++u, ++local) {
-            const int4 tile = p.units[2 * u];
-            const int4 sk = p.units[2 * u + 1];
-            const int kind = sk.z & 0xFF, nh = sk.z >> 8, slot = sk.w & 0xFFFF, nsl = sk.w >> 16;
-            const GemmGroupInfo& gi = p.groups[tile.x];
-            const uint32_t acc = local & 1;
-            const uint32_t acc_phase = (local >> 1) & 1;
-            const int row_local = (int)(q * 32 + lane);
-            const int row = tile.z * S2_BM + (int)rank * 128 + row_local;
-            if (MODE == MODE_UPDATE && kind != 2)
-                prefetch_update_operands(p, gi, tile.y, row,
-                                         tile.w * S2_BN + (nh ? (nh - 1) * 128 + (int)half * 64 : (int)half * 128),
-                                         nh ? 64 : 128);
-            bool ok = mbar_wait(&tfull[acc], acc_phase, abort_flag, p.err, ERR_EPILOGUE);
-            if (kind == 1 && lane == 0) {
-                // the later parts of this split tile, produced first by other clusters
-                for (int sl = 0; sl < nsl && ok; ++sl)
-                    ok = flag_wait(&p.sk_flag[slot + sl], p.epoch, abort_flag, p.err, ERR_SPLIT);
-            }
-            ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0 && ok;
-            if (!__all_sync(0xffffffffu, ok)) break;
-            tc_fence_after();
-            float* sk_row = kind == 0 ? nullptr
-                          : p.sk_partial + (size_t)slot * SK_SLOT_FLOATS + ((size_t)rank * 128 + row_local) * 256;
-            // a column half (nh = 1, 2) has 128 accumulator columns: 2 chunks per warp
-            epilogue_segment<MODE>(p, gi, tile.y, row, tile.w * S2_BN + (nh ? (nh - 1) * 128 : 0),
-                                   tmem_base + acc * ACC_COLS + ((q * 32u) << 16), (int)half * (nh ? 64 : 128), stage,
-                                   kind, sk_row, nsl, nh ? 2 : 4);
-            tc_fence_before();
-            if (kind == 2) __threadfence();
-            __syncwarp();
-            if (lane == 0) {
-                if (kind == 2 && atomicAdd(&p.sk_count[slot], 1) == 2 * NUM_EPI_WARPS - 1) {
-                    // last of the 16 epilogue warps of the pair: the slot is complete
-                    p.sk_count[slot] = 0;
-                    __threadfence();
-                    st_release_gpu(&p.sk_flag[slot], p.epoch);
-                }
-                mbar_arrive_remote(mapa_shared(smem_u32(&tempty[acc]), 0));
-            }
+            pair_epilogue_tma<MODE, ED>(p, rank, h, sE + h * (ED * EU_BUF), ebar + h * 2 * ED,
+                                    ebar + h * 2 * ED + ED, ecoord + h * ED, abort_flag, cid);
         }
     }
 
@@ -1276,9 +1305,11 @@ cudaError_t tc_gemm_prepare() {
     if ((e = cudaFuncSetAttribute(ns_gemm_tc_kernel<MODE_GRAM>, cudaFuncAttributeMaxDynamicSharedMemorySize, S1_SMEM)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ns_gemm_tc_kernel<MODE_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, S1_SMEM)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ns_gemm_tc_kernel<MODE_UPDATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, S1_SMEM)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_GRAM>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM)) != cudaSuccess) return e;
-    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_POLY>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM)) != cudaSuccess) return e;
-    return cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_UPDATE>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2U_SMEM);
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_GRAM, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_POLY, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2U_SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_POLY, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_UPDATE, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2U_SMEM)) != cudaSuccess) return e;
+    return cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_UPDATE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM);
 }
 
 cudaError_t tc_gemm_max_clusters(int* n) {
@@ -1294,23 +1325,32 @@ cudaError_t tc_gemm_max_clusters(int* n) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int nu = 0, ng = 0;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&nu, ns_gemm_tc2_kernel<MODE_UPDATE>, &cfg);
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&nu, ns_gemm_tc2_kernel<MODE_UPDATE, 0>, &cfg);
     if (e != cudaSuccess) return e;
     cfg.dynamicSmemBytes = S2_SMEM;
-    cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-    e = cudaOccupancyMaxActiveClusters(&ng, ns_gemm_tc2_kernel<MODE_GRAM>, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&ng, ns_gemm_tc2_kernel<MODE_GRAM, 1>, &cfg);
     *n = nu < ng ? nu : ng;
     return e;
 }
 
-cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cudaStream_t s) {
+int tc_gemm_var(int mode, int avg_k) {
+    if (mode == MODE_GRAM) return 1;
+    if (mode == MODE_POLY) return avg_k >= 1024 ? 1 : 0;
+    return avg_k >= 2048 ? 1 : 0;
+}
+
+cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cudaStream_t s, int var) {
     if (p.ntiles <= 0) return cudaSuccess;
-    const dim3 g(grid), b(NUM_THREADS);
+    const dim3 g(grid), b(NUM_THREADS), bu(NUM_THREADS_U);
     if (pair) {
         switch (mode) {
-            case MODE_GRAM: return launch_pdl(ns_gemm_tc2_kernel<MODE_GRAM>, g, b, S2_SMEM, s, p);
-            case MODE_POLY: return launch_pdl(ns_gemm_tc2_kernel<MODE_POLY>, g, b, S2_SMEM, s, p);
-            default: return launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE>, g, dim3(NUM_THREADS_U), S2U_SMEM, s, p);
+            case MODE_GRAM: return launch_pdl(ns_gemm_tc2_kernel<MODE_GRAM, 1>, g, bu, S2_SMEM, s, p);
+            case MODE_POLY:
+                return var ? launch_pdl(ns_gemm_tc2_kernel<MODE_POLY, 1>, g, bu, S2_SMEM, s, p)
+                           : launch_pdl(ns_gemm_tc2_kernel<MODE_POLY, 0>, g, bu, S2U_SMEM, s, p);
+            default:
+                return var ? launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE, 1>, g, bu, S2_SMEM, s, p)
+                           : launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE, 0>, g, bu, S2U_SMEM, s, p);
         }
     }
     switch (mode) {

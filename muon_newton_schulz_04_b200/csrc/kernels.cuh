@@ -64,6 +64,11 @@ struct alignas(64) GemmMaps {
     CUtensorMap xe_hi[2];
     CUtensorMap xe_lo_in;
     CUtensorMap xe_lo_out;
+    // GRAM / POLY epilogue of the two-CTA kernel: A and P, [0] the same 128 x 32 box
+    // (64-byte swizzle) for direct stores (and the polynomial's load of A), [1] a
+    // 32 x 128 box (no swizzle) for the mirrored stores of tiles off the diagonal
+    CUtensorMap se_a[2];
+    CUtensorMap se_p[2];
 };
 
 struct GemmGroupInfo {
@@ -117,7 +122,11 @@ int tc_gemm_tile_m(int pair);
 int tc_gemm_tile_n(int pair);
 cudaError_t tc_gemm_prepare();    // sets the dynamic shared-memory attribute once per device
 cudaError_t tc_gemm_max_clusters(int* n);
-cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cudaStream_t s);
+// var: shared-memory configuration of the two-CTA kernel (tc_gemm_var), ignored by the
+// one-CTA kernel
+cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cudaStream_t s, int var = 0);
+// Configuration of a two-CTA launch of `mode` whose tiles have the average K avg_k.
+int tc_gemm_var(int mode, int avg_k);
 
 // Default GEMM variant of new handles and planner queries: the two-CTA kernel unless
 // the environment variable MUON_GEMM_PAIR is "0".
