@@ -174,10 +174,18 @@ UPDATE_TRAFFIC = {
 
 
 def gemm_source_hash() -> str:
+    """Hash of the GEMM kernel's sources with comments and blank lines removed, so
+    that a comment edit does not retire a traffic figure taken on the same code."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in ("gemm_tc.cu", "ptx.cuh", "kernels.cuh"):
-        h.update(open(os.path.join(ROOT, "muon_newton_schulz_04_b200", "csrc", f), "rb").read())
+        text = open(os.path.join(ROOT, "muon_newton_schulz_04_b200", "csrc", f)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for line in text.splitlines():
+            code = line.split("//", 1)[0].strip()
+            if code:
+                h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

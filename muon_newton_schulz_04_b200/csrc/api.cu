@@ -55,6 +55,7 @@ struct Plan {
     // tile lists (tensor-core path)
     int n_gram = 0, n_poly = 0, n_upd = 0;
     int var[3] = {1, 0, 0};              // two-CTA shared-memory configuration per phase
+    bool fused_apply = false;            // bf16 path: the last update also applies W (else the apply kernel)
     // device addresses inside the workspace
     int4* d_tiles_gram = nullptr; int4* d_tiles_poly = nullptr; int4* d_tiles_upd = nullptr;
     // two-CTA kernel: per-phase unit lists (plan.h) and the split-tile partial sums
@@ -406,8 +407,7 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
             sg.rows = d.rows; sg.cols = d.cols; sg.ldn = d.ldn; sg.transposed = d.transposed;
             int nb, na;
             if (d.transposed) {
-                nb = ((d.rows + MT_ROWS - 1) / MT_ROWS) * ((d.cols + MT_COLS - 1) / MT_COLS);
-                na = ((d.rows + EW_TILE - 1) / EW_TILE) * ((d.cols + EW_TILE - 1) / EW_TILE);
+                nb = na = ((d.rows + MT_ROWS - 1) / MT_ROWS) * ((d.cols + MT_COLS - 1) / MT_COLS);
             } else {
                 nb = na = (int)(((long long)d.rows * d.cols + EW_FLAT_ELEMS - 1) / EW_FLAT_ELEMS);
             }
@@ -458,6 +458,7 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
                 P.var[ph] = tc_gemm_var(modes[ph], avg);
             }
         }
+        P.fused_apply = tc_gemm_fused_apply() != 0;
         // nothing is launched with a plan that does not cover its outputs exactly once
         const std::vector<Tile>* lists[3] = {&tg, &tp, &tu};
         for (int ph = 0; ph < 3; ++ph) {
@@ -666,7 +667,7 @@ muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStrea
             gp.units = P.d_units[2]; gp.unit_begin = P.d_unit_begin[2]; gp.epoch = ++h->epoch;
             gp.scale = it == 0 ? P.d_scale : nullptr;
             gp.write_op = (it + 1 < c.ns_steps) ? 1 : 0;
-            if (it + 1 == c.ns_steps) {        // fused apply / copy-out
+            if (it + 1 == c.ns_steps && P.fused_apply) {        // fused apply / copy-out
                 if (hooks && hooks->w_ready) CUDA_TRY(h, cudaStreamWaitEvent(s, hooks->w_ready, 0));
                 gp.apply_mode = copy_out ? 2 : 1;
                 gp.decay = copy_out ? 1.f : 1.f - c.lr * c.weight_decay;
@@ -706,7 +707,7 @@ muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStrea
             }
         }
     }
-    if (bf16 && c.ns_steps > 0) return MUON_OK;
+    if (bf16 && c.ns_steps > 0 && P.fused_apply) return MUON_OK;
     if (hooks && hooks->w_ready) CUDA_TRY(h, cudaStreamWaitEvent(s, hooks->w_ready, 0));
     const float decay = copy_out ? 1.f : 1.f - c.lr * c.weight_decay;
     TIMED(h, 5, s, launch_apply(P.d_segs, P.nmat, P.k7_blocks, decay, c.lr, c.ns_steps == 0 ? P.d_scale : nullptr,

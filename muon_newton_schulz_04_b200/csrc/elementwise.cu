@@ -97,6 +97,24 @@ __device__ __forceinline__ float load_o(const EwSeg& sg, size_t i) {
     return sg.o_src[i];
 }
 
+// Eight consecutive values of O from element i (16-byte aligned for bf16, 32-byte for fp32).
+__device__ __forceinline__ void load_o8(const EwSeg& sg, size_t i, float (&o)[8]) {
+    if (sg.o_hi) {
+        const uint4 h = *reinterpret_cast<const uint4*>(sg.o_hi + i);
+        const uint4 l = sg.o_lo ? *reinterpret_cast<const uint4*>(sg.o_lo + i) : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            o[2 * q] = __uint_as_float(hw[q] << 16) + __uint_as_float(lw[q] << 16);
+            o[2 * q + 1] = __uint_as_float(hw[q] & 0xFFFF0000u) + __uint_as_float(lw[q] & 0xFFFF0000u);
+        }
+    } else {
+        const float4 a = *reinterpret_cast<const float4*>(sg.o_src + i);
+        const float4 b = *reinterpret_cast<const float4*>(sg.o_src + i + 4);
+        o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w; o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+    }
+}
+
 // Copy-out of one value of O to element i of the destination (fp32, or bf16 when
 // the segment asks for it).
 __device__ __forceinline__ void store_out(const EwSeg& sg, float* dst, size_t i, float v) {
@@ -342,7 +360,6 @@ __global__ void __launch_bounds__(EW_THREADS, EW_MIN_BLOCKS) momentum_norm_kerne
 // Apply (copy_out == 0) or copy-out (copy_out == 1) for one block of one matrix.
 __device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay, float lr, const float* o_scale,
                                             int copy_out, float* dst) {
-    __shared__ float tile[EW_TILE][EW_TILE + 1];
     const float os = o_scale ? o_scale[sg.mat] : 1.0f;
     const float step = lr * sg.update_scale;
     if (!sg.transposed) {
@@ -394,24 +411,89 @@ __device__ __forceinline__ void apply_block(const EwSeg& sg, int lb, float decay
             }
         }
     } else {
-        // O = X^T: read X rows j (coalesced over i), write W rows i (coalesced over j)
-        const int tiles_c = (sg.cols + EW_TILE - 1) / EW_TILE;
-        const int i0 = (lb / tiles_c) * EW_TILE, j0 = (lb % tiles_c) * EW_TILE;
-        const int tx = threadIdx.x & 63, ty = threadIdx.x >> 6;
-#pragma unroll 4
-        for (int jj = ty; jj < EW_TILE; jj += 4) {
-            const int j = j0 + jj, i = i0 + tx;
-            tile[jj][tx] = (j < sg.cols && i < sg.rows) ? load_o(sg, (size_t)j * sg.ldn + i) : 0.f;
+        // O = X^T.  Tile of W rows [i0, i0 + MT_ROWS) x cols [j0, j0 + MT_COLS), the
+        // momentum kernel's tile in reverse: O is read along X's rows into
+        // tile_t[j][i], then W is read and written along its own rows, so both sides of
+        // the transpose stay coalesced.
+        __shared__ float tile_t[MT_COLS][MT_ROWS + 1];
+        const int tiles_c = (sg.cols + MT_COLS - 1) / MT_COLS;
+        const int i0 = (lb / tiles_c) * MT_ROWS, j0 = (lb % tiles_c) * MT_COLS;
+        {
+            // thread (ig, jr): X rows jj = jr + 32s, s = 0..3, elements i0 + 8ig .. +7;
+            // 8 lanes cover 64 contiguous elements of a row, all four rows' loads in flight
+            const int ig = threadIdx.x & 7, jr = threadIdx.x >> 3;
+            const int ix = i0 + 8 * ig;
+            float o[MT_COLS / 32][8];
+#pragma unroll
+            for (int sidx = 0; sidx < MT_COLS / 32; ++sidx) {
+                const int jx = j0 + jr + 32 * sidx;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) o[sidx][q] = 0.f;
+                if (jx >= sg.cols || ix >= sg.rows) continue;
+                const size_t xo = (size_t)jx * sg.ldn + ix;
+                if (ix + 7 < sg.rows) load_o8(sg, xo, o[sidx]);
+                else
+                    for (int q = 0; q < 8; ++q)
+                        if (ix + q < sg.rows) o[sidx][q] = load_o(sg, xo + q);
+            }
+#pragma unroll
+            for (int sidx = 0; sidx < MT_COLS / 32; ++sidx)
+#pragma unroll
+                for (int q = 0; q < 8; ++q) tile_t[jr + 32 * sidx][8 * ig + q] = o[sidx][q] * os;
         }
         __syncthreads();
-#pragma unroll 4
-        for (int ii = ty; ii < EW_TILE; ii += 4) {
-            const int i = i0 + ii, j = j0 + tx;
-            if (i < sg.rows && j < sg.cols) {
-                const size_t e = (size_t)i * sg.cols + j;
-                const float o = tile[tx][ii] * os;
-                if (copy_out) store_out(sg, dst, e, o);
-                else dst[e] = fmaf(-step, o, decay * dst[e]);
+        if (sg.vec) {
+            // thread (cg, r): columns j0 + 8cg .. +7 of rows i0 + r + 16p, p = 0..3 (cols % 8
+            // == 0: a group of 8 columns lies wholly inside the matrix or wholly outside)
+            const int cg = threadIdx.x & 15, r = threadIdx.x >> 4;
+            const int j = j0 + 8 * cg;
+            if (j < sg.cols) {
+                float4 wv[MT_ROWS / 16][2];
+                if (!copy_out) {
+#pragma unroll
+                    for (int pp = 0; pp < MT_ROWS / 16; ++pp) {
+                        const int i = i0 + r + 16 * pp;
+                        if (i >= sg.rows) continue;
+                        const float4* wp = reinterpret_cast<const float4*>(dst + (size_t)i * sg.cols + j);
+                        wv[pp][0] = wp[0];
+                        wv[pp][1] = wp[1];
+                    }
+                }
+#pragma unroll
+                for (int pp = 0; pp < MT_ROWS / 16; ++pp) {
+                    const int ir = r + 16 * pp, i = i0 + ir;
+                    if (i >= sg.rows) continue;
+                    float v[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) v[q] = tile_t[8 * cg + q][ir];
+                    const size_t e = (size_t)i * sg.cols + j;
+                    if (copy_out && sg.out_bf16) {
+                        *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(dst) + e) =
+                            make_uint4(pack2_bf16(v[0], v[1]), pack2_bf16(v[2], v[3]), pack2_bf16(v[4], v[5]),
+                                       pack2_bf16(v[6], v[7]));
+                        continue;
+                    }
+                    if (!copy_out) {
+                        const float w8[8] = {wv[pp][0].x, wv[pp][0].y, wv[pp][0].z, wv[pp][0].w,
+                                             wv[pp][1].x, wv[pp][1].y, wv[pp][1].z, wv[pp][1].w};
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) v[q] = fmaf(-step, v[q], decay * w8[q]);
+                    }
+                    float4* wp = reinterpret_cast<float4*>(dst + e);
+                    wp[0] = make_float4(v[0], v[1], v[2], v[3]);
+                    wp[1] = make_float4(v[4], v[5], v[6], v[7]);
+                }
+            }
+        } else {
+            // consecutive threads take consecutive columns of a row of W
+            for (int e = threadIdx.x; e < MT_ROWS * MT_COLS; e += EW_THREADS) {
+                const int ii = e / MT_COLS, jj = e % MT_COLS;
+                const int i = i0 + ii, j = j0 + jj;
+                if (i >= sg.rows || j >= sg.cols) continue;
+                const size_t we = (size_t)i * sg.cols + j;
+                const float o = tile_t[jj][ii];
+                if (copy_out) store_out(sg, dst, we, o);
+                else dst[we] = fmaf(-step, o, decay * dst[we]);
             }
         }
     }
@@ -437,7 +519,7 @@ __global__ void __launch_bounds__(EW_THREADS) copy_out_one_kernel(const EwSeg sg
 // rows c, c + RMS_CHUNKS, ... of the matrix's oriented m x n iterate in fp64;
 // update_rms_finish_kernel adds the RMS_CHUNKS partials of each matrix in a fixed
 // order, so the result is bitwise reproducible.
-constexpr int RMS_CHUNKS = 32;
+constexpr int RMS_CHUNKS = UPDATE_RMS_PARTIALS;
 
 __global__ void __launch_bounds__(EW_THREADS) update_sq_kernel(const EwSeg* __restrict__ segs,
                                                                const float* __restrict__ o_scale,
@@ -449,9 +531,26 @@ __global__ void __launch_bounds__(EW_THREADS) update_sq_kernel(const EwSeg* __re
     const int m = sg.transposed ? sg.cols : sg.rows, n = sg.transposed ? sg.rows : sg.cols;
     const float os = o_scale ? o_scale[sg.mat] : 1.0f;
     double acc = 0.0;
+    // bf16 pair with 16-byte rows (ldn is a multiple of 8): 8 elements per load
+    const bool vec = sg.o_hi != nullptr && sg.o_lo != nullptr && sg.ldn % 8 == 0;
+    const int n8 = vec ? n / 8 : 0;
     for (int r = blockIdx.x; r < m; r += RMS_CHUNKS) {
-        for (int c = threadIdx.x; c < n; c += EW_THREADS) {
-            const double v = (double)(load_o(sg, (size_t)r * sg.ldn + c) * os);
+        const size_t row = (size_t)r * sg.ldn;
+        for (int c8 = threadIdx.x; c8 < n8; c8 += EW_THREADS) {
+            const uint4 hv = __ldcs(reinterpret_cast<const uint4*>(sg.o_hi + row) + c8);
+            const uint4 lv = __ldcs(reinterpret_cast<const uint4*>(sg.o_lo + row) + c8);
+            const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                const float2 h2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[t]));
+                const float2 l2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lw[t]));
+                const double v0 = (double)((h2.x + l2.x) * os), v1 = (double)((h2.y + l2.y) * os);
+                acc += v0 * v0;
+                acc += v1 * v1;
+            }
+        }
+        for (int c = 8 * n8 + threadIdx.x; c < n; c += EW_THREADS) {
+            const double v = (double)(load_o(sg, row + c) * os);
             acc += v * v;
         }
     }
@@ -459,20 +558,19 @@ __global__ void __launch_bounds__(EW_THREADS) update_sq_kernel(const EwSeg* __re
     if (threadIdx.x == 0) part[(size_t)blockIdx.y * RMS_CHUNKS + blockIdx.x] = tot;
 }
 
-__global__ void __launch_bounds__(32) update_rms_finish_kernel(const EwSeg* __restrict__ segs,
-                                                               const double* __restrict__ part, float lr,
-                                                               float* __restrict__ rms) {
+__global__ void __launch_bounds__(EW_THREADS) update_rms_finish_kernel(const EwSeg* __restrict__ segs,
+                                                                       const double* __restrict__ part, float lr,
+                                                                       float* __restrict__ rms) {
+    __shared__ double red[EW_THREADS / 32];
     pdl_trigger();
     pdl_wait();
     const EwSeg sg = segs[blockIdx.x];
-    double v = part[(size_t)blockIdx.x * RMS_CHUNKS + threadIdx.x];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+    const double v = block_sum(part[(size_t)blockIdx.x * RMS_CHUNKS + threadIdx.x], red);
     if (threadIdx.x == 0)
         rms[blockIdx.x] = (float)((double)lr * fabs((double)sg.update_scale) *
                                   sqrt(v / ((double)sg.rows * (double)sg.cols)));
 }
-static_assert(RMS_CHUNKS == 32, "the finish kernel reduces one warp");
+static_assert(RMS_CHUNKS == EW_THREADS, "the finish kernel reduces one partial per thread");
 
 }  // namespace
 
@@ -481,7 +579,7 @@ cudaError_t launch_update_rms(const EwSeg* segs, int nseg, const float* o_scale,
     if (nseg <= 0) return cudaSuccess;
     cudaError_t e = launch_pdl(update_sq_kernel, dim3(RMS_CHUNKS, nseg), dim3(EW_THREADS), 0, s, segs, o_scale, part);
     if (e != cudaSuccess) return e;
-    return launch_pdl(update_rms_finish_kernel, dim3(nseg), dim3(32), 0, s, segs, (const double*)part, lr, rms);
+    return launch_pdl(update_rms_finish_kernel, dim3(nseg), dim3(EW_THREADS), 0, s, segs, (const double*)part, lr, rms);
 }
 
 cudaError_t launch_momentum_norm(const EwSeg* segs, int nseg, int nblocks, double* partials, float mu,

@@ -6,12 +6,13 @@
 //
 //   GRAM    A  = alpha * X X^T            (upper-triangle tiles, mirrored)
 //   POLY    P  = b*A + c * A A            (A symmetric: A A = A A^T; upper tiles, mirrored)
-//   UPDATE  X' = alpha * P X + beta * X   (the aX term in the epilogue, X read in fp32)
+//   UPDATE  X' = alpha * P X + beta * X   (the aX term in the epilogue; X = hi + lo, the
+//                                         bf16 pair, read and written by the epilogue)
 //
 // On the first step alpha/beta absorb the Frobenius normalisation s = 1/(||U||+eps):
 // A0 = s^2 UU^T and X1 = s P U + a s U.
 //
-// Two kernels share the epilogue:
+// Two kernels:
 //
 //  ns_gemm_tc_kernel (one CTA per tile, 128 x 256 tiles), 320 threads:
 //   warp 0      TMA producer: 4-stage ring of (128x64 A-operand, 256x64 B-operand)
@@ -19,19 +20,28 @@
 //   warp 1      allocates 512 TMEM columns (two 128x256 fp32 accumulators) and issues
 //               tcgen05.mma kind::f16 (M=128, N=256, K=16) from one thread.
 //   warps 2-9   epilogue: tcgen05.ld of the accumulator (each warp owns the 32 TMEM
-//               lanes its rank allows and half of the columns), scale, residual, store.
+//               lanes its rank allows and half of the columns), scale, residual, and
+//               stores through the load/store units.
 //
-//  ns_gemm_tc2_kernel (a cluster of two CTAs per 256 x 256 tile): each CTA stages its
-//   128 rows of A and its 128 columns of B (6-stage ring of 16 + 16 KiB), the even CTA
-//   issues tcgen05.mma.cta_group::2 (M=256, N=256) which reads both CTAs' shared memory,
-//   and each CTA's TMEM receives its 128 accumulator rows.  Per SM this moves half the
-//   B-operand bytes of the one-CTA tile through shared memory.  The odd CTA's TMA
-//   loads complete on the even CTA's barrier; MMA completion is committed to the
-//   barriers of both CTAs by address; no multicast form is used.
+//  ns_gemm_tc2_kernel (a cluster of two CTAs per 256 x 256 tile), 384 threads per CTA:
+//   warp 0      TMA producer: each CTA stages its 128 rows of A and its 128 columns of B
+//               (a ring of 4 or 5 stages of 16 + 16 KiB); the odd CTA's loads complete
+//               on the even CTA's barrier; no multicast form is used.
+//   warp 1      the even CTA's elected thread issues tcgen05.mma.cta_group::2 (M=256,
+//               N=256, K=16), which reads both CTAs' shared memory; each CTA's TMEM
+//               receives its 128 accumulator rows; completion is committed to the
+//               barriers of both CTAs by address.
+//   warps 2-9   epilogue compute: two column halves of four warps; tcgen05.ld, then
+//               the mode's arithmetic on 128 x 32 boxes in shared memory.
+//   warps 10-11 epilogue TMA, one per column half: load the boxes the epilogue reads
+//               (X = hi + lo for UPDATE, A for POLY) ahead of time and store the
+//               finished boxes with bulk tensor stores.
+//   Per SM this moves half the B-operand bytes of the one-CTA tile through shared
+//   memory, and the epilogue's global traffic leaves the load/store units.
 //
 // The double-buffered accumulator lets the epilogue of tile i overlap the main
-// loop of tile i+1.  Tiles are taken round-robin from a cost-sorted list that
-// spans all matrices of the call, so many small matrices fill the 148 SMs.
+// loop of tile i+1.  Tiles are taken from per-cluster lists built from a cost-sorted
+// list that spans all matrices of the call, so many small matrices fill the 148 SMs.
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -594,38 +604,46 @@ __device__ __forceinline__ void apply_row(const GemmParams& p, const GemmGroupIn
         }
         return;
     }
+    // every load of W is issued before the first store: with the stores in between,
+    // the compiler cannot tell that the addresses differ and waits out each load
     if (!sg.transposed) {
         float* wr = w + (size_t)row * sg.cols;
         if (sg.vec && col0 + NC - 1 < gi.n) {
             float4* w4 = reinterpret_cast<float4*>(wr + col0);
+            float4 x[NC / 4];
+            if (!copy) {
+#pragma unroll
+                for (int qq = 0; qq < NC / 4; ++qq) x[qq] = __ldcg(w4 + qq);
+            }
 #pragma unroll
             for (int qq = 0; qq < NC / 4; ++qq) {
                 float4 o = make_float4(val[4 * qq], val[4 * qq + 1], val[4 * qq + 2], val[4 * qq + 3]);
                 if (!copy) {
-                    const float4 x = w4[qq];
-                    o.x = fmaf(-step, o.x, p.decay * x.x);
-                    o.y = fmaf(-step, o.y, p.decay * x.y);
-                    o.z = fmaf(-step, o.z, p.decay * x.z);
-                    o.w = fmaf(-step, o.w, p.decay * x.w);
+                    o.x = fmaf(-step, o.x, p.decay * x[qq].x);
+                    o.y = fmaf(-step, o.y, p.decay * x[qq].y);
+                    o.z = fmaf(-step, o.z, p.decay * x[qq].z);
+                    o.w = fmaf(-step, o.w, p.decay * x[qq].w);
                 }
                 w4[qq] = o;
             }
         } else {
+            float x[NC];
 #pragma unroll
-            for (int j = 0; j < NC; ++j) {
-                const int c = col0 + j;
-                if (c < gi.n) wr[c] = copy ? val[j] : fmaf(-step, val[j], p.decay * wr[c]);
-            }
+            for (int j = 0; j < NC; ++j) x[j] = (!copy && col0 + j < gi.n) ? __ldcg(wr + col0 + j) : 0.f;
+#pragma unroll
+            for (int j = 0; j < NC; ++j)
+                if (col0 + j < gi.n) wr[col0 + j] = copy ? val[j] : fmaf(-step, val[j], p.decay * x[j]);
         }
     } else {
+        // W[c][row]: lanes hold consecutive rows, so each access of the warp is coalesced
+        float x[NC];
 #pragma unroll
-        for (int j = 0; j < NC; ++j) {
-            const int c = col0 + j;
-            if (c < gi.n) {
-                float* wp = w + (size_t)c * sg.cols + row;
-                *wp = copy ? val[j] : fmaf(-step, val[j], p.decay * *wp);
-            }
-        }
+        for (int j = 0; j < NC; ++j)
+            x[j] = (!copy && col0 + j < gi.n) ? __ldcg(w + (size_t)(col0 + j) * sg.cols + row) : 0.f;
+#pragma unroll
+        for (int j = 0; j < NC; ++j)
+            if (col0 + j < gi.n)
+                w[(size_t)(col0 + j) * sg.cols + row] = copy ? val[j] : fmaf(-step, val[j], p.decay * x[j]);
     }
 }
 

@@ -155,8 +155,8 @@ cudaError_t launch_apply(const EwSeg* segs, int nseg, int nblocks, float decay, 
                          const float* o_scale, int copy_out, cudaStream_t s);
 cudaError_t launch_copy_out_one(const EwSeg& seg, float* dst, const float* o_scale, cudaStream_t s);
 // Per matrix: rms[i] = lr * |s_i| * sqrt(sum of O_i^2 / (rows * cols)) over the final
-// iterate; `part` holds 32 doubles per matrix (fixed-order partial sums).
-constexpr int UPDATE_RMS_PARTIALS = 32;
+// iterate; `part` holds UPDATE_RMS_PARTIALS doubles per matrix (fixed-order partial sums).
+constexpr int UPDATE_RMS_PARTIALS = 256;
 cudaError_t launch_update_rms(const EwSeg* segs, int nseg, const float* o_scale, float lr, double* part, float* rms,
                               cudaStream_t s);
 // QK-Clip: rows of head h of W_q and W_k (n_heads * head_dim rows, `cols` columns)
@@ -184,7 +184,7 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 constexpr int EW_THREADS = 256;
 constexpr int EW_FLAT_ELEMS = 8192;      // elements per block on the flat path
-constexpr int EW_TILE = 64;              // transpose tile edge of the apply kernel
-constexpr int MT_ROWS = 64, MT_COLS = 128;   // transpose tile of the momentum kernel (rows x cols of W)
+// transpose tile of the momentum and apply kernels for tall matrices (rows x cols of W)
+constexpr int MT_ROWS = 64, MT_COLS = 128;
 
 }  // namespace muon

@@ -208,6 +208,11 @@ int tc_gemm_split_tiles() {
     return (v && std::strcmp(v, "1") == 0) ? 1 : 0;
 }
 
+int tc_gemm_fused_apply() {
+    const char* v = std::getenv("MUON_FUSED_APPLY");
+    return (v && std::strcmp(v, "1") == 0) ? 1 : 0;
+}
+
 int tc_gemm_default_pair() {
     const char* v = std::getenv("MUON_GEMM_PAIR");
     return (v && std::strcmp(v, "0") == 0) ? 0 : 1;
