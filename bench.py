@@ -169,7 +169,7 @@ def update_gemm_flops(w: wl.Workload):
 # has no counters until it is captured again.
 UPDATE_TRAFFIC = {
     # (source hash, workload key, variant) -> bytes per launch
-    ("08b7a847eda86a7f", "square4096", "pair"): 162.974e6,     # profiles/ns_gemm_update_square4096.md
+    ("c823c1b316181391", "square4096", "pair"): 171.683e6,     # profiles/ns_gemm_square4096.md
 }
 
 

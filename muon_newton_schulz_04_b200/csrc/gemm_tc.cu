@@ -101,11 +101,16 @@ static_assert(EU_COLS == 32 || EU_COLS == 64, "epilogue chunks are 32 or 64 colu
 constexpr int EU_ROWS = 128;                        // rows per chunk: the CTA's accumulator rows
 constexpr int EU_DEPTH = MUON_EU_DEPTH;            // update epilogue ring depth
 constexpr int ES_DEPTH = MUON_ES_DEPTH;            // ring depth of the long-K configuration
-// Two shared-memory configurations of the two-CTA kernel: VAR 0 (ring depth EU_DEPTH,
-// S2U_STAGES operand stages) for short K, VAR 1 (ES_DEPTH, S2S_STAGES) for long K.
-// The Gram always takes VAR 1 (its epilogue loads nothing); the polynomial and the
-// update choose per launch from the plan's K (launch_tc_gemm's `var`).
-__host__ __device__ constexpr int eu_depth(int var) { return var ? ES_DEPTH : EU_DEPTH; }
+// Three shared-memory configurations of the two-CTA kernel: VAR 0 (ring depth EU_DEPTH,
+// S2U_STAGES operand stages) for short K, VAR 1 (ES_DEPTH, S2S_STAGES) for long K and
+// VAR 2 (one epilogue buffer per half, S2L_STAGES operand stages) for the longest K,
+// where a tile's main loop leaves the epilogue enough time to run one chunk at a time.
+// Each launch takes the one tc_gemm_var picks from the plan's K.
+#ifndef MUON_S2L_STAGES
+#define MUON_S2L_STAGES 6
+#endif
+constexpr int S2L_STAGES = MUON_S2L_STAGES;
+__host__ __device__ constexpr int eu_depth(int var) { return var == 2 ? 1 : var ? ES_DEPTH : EU_DEPTH; }
 constexpr int EU_ROW_BYTES = EU_COLS * 2;
 constexpr int EU_BOX = EU_ROWS * EU_ROW_BYTES;      // 8 KiB
 constexpr int EU_BUF = 2 * EU_BOX;                  // hi + lo
@@ -116,7 +121,7 @@ static_assert(EU_DEPTH >= 2 && EU_DEPTH <= 6 && ES_DEPTH >= 2 && ES_DEPTH <= 6, 
 
 // Every mode of the two-CTA kernel uses the TMA epilogue (the Gram and polynomial
 // products store their symmetric output through the same ring of boxes).
-constexpr int s2_stages(int var) { return var ? S2S_STAGES : S2U_STAGES; }
+constexpr int s2_stages(int var) { return var == 2 ? S2L_STAGES : var ? S2S_STAGES : S2U_STAGES; }
 constexpr int s2_epi_bytes(int var) { return 2 * eu_depth(var) * EU_BUF; }
 constexpr int s2_threads(int) { return NUM_THREADS_U; }
 // barriers: full / empty per stage, two tfull / tempty, drain, the epilogue ring's
@@ -131,7 +136,8 @@ constexpr int s2_smem(int var) {
 }
 constexpr int S2_SMEM = s2_smem(1);
 constexpr int S2U_SMEM = s2_smem(0);
-static_assert(S1_SMEM <= 232448 && S2_SMEM <= 232448 && S2U_SMEM <= 232448,
+constexpr int S2L_SMEM = s2_smem(2);
+static_assert(S1_SMEM <= 232448 && S2_SMEM <= 232448 && S2U_SMEM <= 232448 && S2L_SMEM <= 232448,
               "dynamic shared memory above the 227 KiB limit");
 static_assert((s2_stages(0) * (S2_A + S2_B)) % 1024 == 0 && (s2_stages(1) * (S2_A + S2_B)) % 1024 == 0 &&
               EU_BUF % 1024 == 0, "buffer alignment");
@@ -940,9 +946,10 @@ __device__ __forceinline__ void sym_compute(uint32_t d_s, uint32_t t_s, int lane
 
 // The TMA warp of one column half of the two-CTA epilogue (one elected
 // thread): walks the half's load chunks of every unit of its cluster in order,
-// loading chunk j + EU_DEPTH - 1 into the ring once chunk j - 1's stores have read
-// their buffer, and storing chunk j once the half's four compute warps have arrived
-// on its done barrier.  Returns false when a bounded wait gave up.
+// loading chunk j + D - 1 into the ring once chunk j - 1's stores have read
+// their buffer (with a ring of one buffer: chunk j + 1 once chunk j's stores have),
+// and storing chunk j once the half's four compute warps have arrived on its done
+// barrier.  Returns false when a bounded wait gave up.
 template <int MODE, int D>
 __device__ __forceinline__ bool pair_epilogue_tma(const GemmParams& p, uint32_t rank, int half, uint8_t* ebuf,
                                                   uint64_t* efull, uint64_t* edone, int4* coord,
@@ -954,10 +961,12 @@ __device__ __forceinline__ bool pair_epilogue_tma(const GemmParams& p, uint32_t 
     // coord[b]: (group, matrix, row0, col0) of the chunk in buffer b (shared memory)
     uint32_t issued = 0, stored = 0;
     bool more = true, ok = true;
+    // store groups that may still be reading their buffer after the wait below
+    constexpr uint32_t WR = D > 1 ? 1u : 0u;
     while (true) {
         // load chunk i once the stores of chunk i - D have read its buffer: after
-        // the wait below, every store but the last one has
-        while (more && issued + 1 < stored + D) {
+        // the wait below, every store but the last WR ones has
+        while (more && issued + WR < stored + D) {
             if (ic >= inch) {
                 if (++iu >= u_end) { more = false; break; }
                 itile = p.units[2 * iu];
@@ -1003,7 +1012,7 @@ __device__ __forceinline__ bool pair_epilogue_tma(const GemmParams& p, uint32_t 
         }
         bulk_commit();
         ++stored;
-        bulk_wait_read<1>();              // every store but this one has read its buffer
+        bulk_wait_read<WR>();             // every store but the last WR ones has read its buffer
     }
     bulk_wait_all();
     // loads still in flight (after an abort) must land before the CTA retires
@@ -1310,8 +1319,6 @@ ns_gemm_tc2_kernel(const __grid_constant__ GemmParams p) {
 
 }  // namespace
 
-size_t tc_gemm_smem_bytes(int pair) { return pair ? S2_SMEM : S1_SMEM; }
-size_t tc_gemm_smem_bytes_mode(int mode, int pair) { return pair ? (size_t)s2_smem(mode) : (size_t)S1_SMEM; }
 int tc_gemm_epi_cols() { return EU_COLS; }
 int tc_gemm_epi_rows() { return EU_ROWS; }
 int tc_gemm_threads() { return NUM_THREADS; }
@@ -1327,7 +1334,10 @@ cudaError_t tc_gemm_prepare() {
     if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_POLY, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2U_SMEM)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_POLY, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM)) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_UPDATE, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2U_SMEM)) != cudaSuccess) return e;
-    return cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_UPDATE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM);
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_UPDATE, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2_SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_GRAM, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2L_SMEM)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_POLY, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2L_SMEM)) != cudaSuccess) return e;
+    return cudaFuncSetAttribute(ns_gemm_tc2_kernel<MODE_UPDATE, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, S2L_SMEM);
 }
 
 cudaError_t tc_gemm_max_clusters(int* n) {
@@ -1351,10 +1361,21 @@ cudaError_t tc_gemm_max_clusters(int* n) {
     return e;
 }
 
+// average K from which a phase takes VAR 2 (the deepest operand ring)
+#ifndef MUON_GRAM_VAR2_K
+#define MUON_GRAM_VAR2_K (1 << 30)
+#endif
+#ifndef MUON_POLY_VAR2_K
+#define MUON_POLY_VAR2_K (1 << 30)
+#endif
+#ifndef MUON_UPD_VAR2_K
+#define MUON_UPD_VAR2_K 3072
+#endif
+
 int tc_gemm_var(int mode, int avg_k) {
-    if (mode == MODE_GRAM) return 1;
-    if (mode == MODE_POLY) return avg_k >= 1024 ? 1 : 0;
-    return avg_k >= 2048 ? 1 : 0;
+    if (mode == MODE_GRAM) return avg_k >= MUON_GRAM_VAR2_K ? 2 : 1;
+    if (mode == MODE_POLY) return avg_k >= MUON_POLY_VAR2_K ? 2 : avg_k >= 1024 ? 1 : 0;
+    return avg_k >= MUON_UPD_VAR2_K ? 2 : avg_k >= 2048 ? 1 : 0;
 }
 
 cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cudaStream_t s, int var) {
@@ -1362,13 +1383,17 @@ cudaError_t launch_tc_gemm(int mode, int pair, const GemmParams& p, int grid, cu
     const dim3 g(grid), b(NUM_THREADS), bu(NUM_THREADS_U);
     if (pair) {
         switch (mode) {
-            case MODE_GRAM: return launch_pdl(ns_gemm_tc2_kernel<MODE_GRAM, 1>, g, bu, S2_SMEM, s, p);
+            case MODE_GRAM:
+                return var == 2 ? launch_pdl(ns_gemm_tc2_kernel<MODE_GRAM, 2>, g, bu, S2L_SMEM, s, p)
+                                : launch_pdl(ns_gemm_tc2_kernel<MODE_GRAM, 1>, g, bu, S2_SMEM, s, p);
             case MODE_POLY:
-                return var ? launch_pdl(ns_gemm_tc2_kernel<MODE_POLY, 1>, g, bu, S2_SMEM, s, p)
-                           : launch_pdl(ns_gemm_tc2_kernel<MODE_POLY, 0>, g, bu, S2U_SMEM, s, p);
+                return var == 2 ? launch_pdl(ns_gemm_tc2_kernel<MODE_POLY, 2>, g, bu, S2L_SMEM, s, p)
+                     : var      ? launch_pdl(ns_gemm_tc2_kernel<MODE_POLY, 1>, g, bu, S2_SMEM, s, p)
+                                : launch_pdl(ns_gemm_tc2_kernel<MODE_POLY, 0>, g, bu, S2U_SMEM, s, p);
             default:
-                return var ? launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE, 1>, g, bu, S2_SMEM, s, p)
-                           : launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE, 0>, g, bu, S2U_SMEM, s, p);
+                return var == 2 ? launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE, 2>, g, bu, S2L_SMEM, s, p)
+                     : var      ? launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE, 1>, g, bu, S2_SMEM, s, p)
+                                : launch_pdl(ns_gemm_tc2_kernel<MODE_UPDATE, 0>, g, bu, S2U_SMEM, s, p);
         }
     }
     switch (mode) {

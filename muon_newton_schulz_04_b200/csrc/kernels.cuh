@@ -110,14 +110,12 @@ struct GemmParams {
 // One partial-sum slot: both CTAs' 128 x 256 fp32 accumulator halves.
 constexpr int SK_SLOT_FLOATS = 2 * 128 * 256;
 
-// pair = 1: the two-CTA kernel (256 x 256 tiles, grid = 2 x clusters);
-// pair = 0: the one-CTA kernel (128 x 256 tiles).
-size_t tc_gemm_smem_bytes(int pair);
-size_t tc_gemm_smem_bytes_mode(int mode, int pair);
 // box of the two-CTA UPDATE epilogue: rows x columns (128 x 32 bf16)
 int tc_gemm_epi_cols();
 int tc_gemm_epi_rows();
 int tc_gemm_threads();
+// pair = 1: the two-CTA kernel (256 x 256 tiles, grid = 2 x clusters);
+// pair = 0: the one-CTA kernel (128 x 256 tiles).
 int tc_gemm_tile_m(int pair);
 int tc_gemm_tile_n(int pair);
 cudaError_t tc_gemm_prepare();    // sets the dynamic shared-memory attribute once per device

@@ -75,9 +75,9 @@ int tc_gemm_split_tiles();
 // 0 unless the environment variable MUON_FUSED_APPLY is "1".  With 1 the bf16 path
 // applies W <- decay*W - lr*s*O (or copies O out) in the epilogue of the last update
 // GEMM; by default the update GEMM only writes O and the apply kernel does the rest.
-// The fused form moves 4 B/elem less but measured slower on every workload with
-// small matrices (the epilogue warps, one matrix row per lane, wait on W's reads
-// while the accumulator they hold stalls the MMAs).
+// The fused form moves 4 B/elem less but measured slower on the GPT-2 and 4096^2
+// workloads (its epilogue warps, one matrix row per lane, wait on W's reads while the
+// accumulator they hold stalls the MMAs) and within noise on the MoE one.
 int tc_gemm_fused_apply();
 
 // 1 unless the environment variable MUON_GEMM_PAIR is "0" (see kernels.cuh).
