@@ -84,9 +84,8 @@ constexpr int S2_B = 128 * BK * 2;            // 16 KiB: this CTA's 128 columns 
 #ifndef MUON_S2U_STAGES
 #define MUON_S2U_STAGES 4
 #endif
-// Gram: the epilogue loads nothing, so a ring of two boxes suffices and the operand
-// ring gets a fifth stage for its long K (n); the polynomial (K = m, A loaded for the
-// b*A term) keeps the update's ring and stages.
+// Long K (polynomial from K = 1024, update from K = 2048): a ring of two boxes per
+// half and a fifth operand stage.
 #ifndef MUON_ES_DEPTH
 #define MUON_ES_DEPTH 2
 #endif
@@ -1355,15 +1354,18 @@ cudaError_t tc_gemm_max_clusters(int* n) {
     int nu = 0, ng = 0;
     cudaError_t e = cudaOccupancyMaxActiveClusters(&nu, ns_gemm_tc2_kernel<MODE_UPDATE, 0>, &cfg);
     if (e != cudaSuccess) return e;
-    cfg.dynamicSmemBytes = S2_SMEM;
-    e = cudaOccupancyMaxActiveClusters(&ng, ns_gemm_tc2_kernel<MODE_GRAM, 1>, &cfg);
+    cfg.dynamicSmemBytes = S2L_SMEM;
+    e = cudaOccupancyMaxActiveClusters(&ng, ns_gemm_tc2_kernel<MODE_GRAM, 2>, &cfg);
     *n = nu < ng ? nu : ng;
     return e;
 }
 
-// average K from which a phase takes VAR 2 (the deepest operand ring)
+// average K from which a phase takes VAR 2 (the deepest operand ring).  The Gram's
+// epilogue loads nothing, so it takes VAR 2 at every K (measured 1-2 % faster than
+// VAR 1 on the GPT-2 and MoE workloads, equal at 4096^2); for the polynomial and
+// the update a one-buffer ring is only good when a tile's main loop is long.
 #ifndef MUON_GRAM_VAR2_K
-#define MUON_GRAM_VAR2_K (1 << 30)
+#define MUON_GRAM_VAR2_K 0
 #endif
 #ifndef MUON_POLY_VAR2_K
 #define MUON_POLY_VAR2_K (1 << 30)
