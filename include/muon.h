@@ -294,15 +294,14 @@ const char* muon_status_string(muon_status s);
  * device array of MUON_NOALLOC_MAX_BLOCKS doubles (512 KiB) that every GPU which
  * loads the library holds until the process exits; a matrix of more than
  * MUON_NOALLOC_MAX_BLOCKS * 8192 elements is rejected with MUON_ERR_UNSUPPORTED.
- * The first call on a device looks up the array's device address
- * (cudaGetSymbolAddress) and keeps it for the life of the process, so make that
- * first call before any stream capture.  With the CUDA runtime's lazy module
- * loading (the default since CUDA 12) that first call is also when the module is
- * loaded and the 512 KiB are reserved on the device: make it a warm-up call while
- * device memory is still available.  After cudaDeviceReset on a device the kept
- * address is stale; do not use this entry point on that device again in the
- * process.  B, U_out and norm_out are written, so none of them may overlap another
- * buffer of the call (MUON_ERR_INVALID).
+ * Every call looks up the array's device address (cudaGetSymbolAddress) on the
+ * current device, so the address stays right after cudaDeviceReset or a new
+ * primary context.  With the CUDA runtime's lazy module loading (the default since
+ * CUDA 12) the first call on a device (and the first after a reset) is when the
+ * module is loaded and the 512 KiB are reserved on the device: make it a warm-up
+ * call while device memory is still available and before any stream capture.
+ * B, U_out and norm_out are written, so none of them may overlap another buffer
+ * of the call (MUON_ERR_INVALID).
  * All calls share the one array, and each call overwrites the partial sums it
  * reads: calls whose work overlaps on the GPU (unordered streams) race and give
  * wrong norms.  err_msg (optional host buffer of err_cap bytes) receives a

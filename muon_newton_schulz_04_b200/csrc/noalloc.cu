@@ -11,12 +11,13 @@
 // that loads the library holds it until the process exits.
 //
 // The array's name in host code is a host-side stand-in, not a device address,
-// so the entry point looks the address up once per device with
-// cudaGetSymbolAddress (with that device current) and passes it to the kernels.
+// so every call looks the address up with cudaGetSymbolAddress (with the device
+// current) and passes it to the kernels.  The lookup is not cached: after a
+// cudaDeviceReset or a new primary context the module is loaded again, possibly at
+// another address.
 #include <cuda_runtime.h>
 
 #include <cstdio>
-#include <mutex>
 
 #include "../../include/muon.h"
 #include "kernels.cuh"
@@ -29,9 +30,6 @@ constexpr int NA_ELEMS_PER_BLOCK = 8192;   // 256 threads x 8 elements x 4 round
 
 static __device__ __align__(256) double g_noalloc_partials[MUON_NOALLOC_MAX_BLOCKS];
 
-constexpr int NA_MAX_DEVICES = 64;
-std::mutex g_setup_mutex;
-double* g_scratch_addr[NA_MAX_DEVICES] = {};
 
 __device__ __forceinline__ double na_block_sum(double v, double* red) {
 #pragma unroll
@@ -122,27 +120,16 @@ extern "C" muon_status muon_momentum_norm_noalloc(int rows, int cols, int grad_d
         put_msg(err_msg, err_cap, "B, U_out and norm_out are written: they may not overlap each other or G");
         return MUON_ERR_INVALID;
     }
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= NA_MAX_DEVICES) {
-        cudaGetLastError();
-        put_msg(err_msg, err_cap, "no usable current CUDA device");
-        return MUON_ERR_CUDA;
-    }
-    double* scratch = nullptr;
+    void* p = nullptr;
     {
-        std::lock_guard<std::mutex> lock(g_setup_mutex);
-        if (!g_scratch_addr[dev]) {
-            void* p = nullptr;
-            cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_partials);
-            if (e != cudaSuccess || !p) {
-                cudaGetLastError();
-                put_msg(err_msg, err_cap, "cudaGetSymbolAddress of the static scratch failed");
-                return MUON_ERR_CUDA;
-            }
-            g_scratch_addr[dev] = static_cast<double*>(p);
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+        if (e != cudaSuccess || !p) {
+            cudaGetLastError();
+            put_msg(err_msg, err_cap, "cudaGetSymbolAddress of the static scratch failed");
+            return MUON_ERR_CUDA;
         }
-        scratch = g_scratch_addr[dev];
     }
+    double* scratch = static_cast<double*>(p);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     momentum_norm_noalloc_kernel<<<(unsigned)nblocks, NA_THREADS, 0, s>>>(G, grad_dtype == MUON_BF16 ? 1 : 0, B, U_out,
                                                                          total, momentum, nesterov, scratch);
