@@ -3,8 +3,9 @@
 // Muon step ("Muon: An optimizer for hidden layers in neural networks",
 // section 4):
 //
-//   momentum_norm  ->  ns_steps x (GRAM -> POLY -> UPDATE)
-//   (the last UPDATE applies W; the fp32 debug path and ns_steps = 0 use the apply kernel)
+//   momentum_norm  ->  ns_steps x (GRAM -> POLY -> UPDATE)  ->  apply
+//   (with MUON_FUSED_APPLY=1 the bf16 path's last UPDATE applies W in its epilogue
+//   and no apply kernel runs)
 //
 // All launches go to the caller's stream; nothing here synchronises except the
 // entry points documented to do so.
@@ -666,7 +667,6 @@ muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStrea
             gp.tiles = P.d_tiles_upd; gp.ntiles = P.n_upd; gp.alpha = 1.f; gp.beta = c.ns_a;
             gp.units = P.d_units[2]; gp.unit_begin = P.d_unit_begin[2]; gp.epoch = ++h->epoch;
             gp.scale = it == 0 ? P.d_scale : nullptr;
-            gp.write_op = (it + 1 < c.ns_steps) ? 1 : 0;
             if (it + 1 == c.ns_steps && P.fused_apply) {        // fused apply / copy-out
                 if (hooks && hooks->w_ready) CUDA_TRY(h, cudaStreamWaitEvent(s, hooks->w_ready, 0));
                 gp.apply_mode = copy_out ? 2 : 1;
@@ -1233,7 +1233,6 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     gp.alpha = a->alpha;
     gp.beta = a->beta;
     gp.scale = nullptr;
-    gp.write_op = (phase == MUON_NS_UPDATE && a->out_op) ? 1 : 0;
     gp.err = h->d_err;
     const int mode = phase == MUON_NS_GRAM ? MODE_GRAM : phase == MUON_NS_POLY ? MODE_POLY : MODE_UPDATE;
     CUDA_TRY(h, launch_tc_gemm(mode, h->pair, gp, gemm_grid(h, gp.ntiles), s,
