@@ -149,10 +149,13 @@ def elementwise_bytes(w: wl.Workload):
     B (4 B) and the bf16 iterate X0 (2 B) = 12 B/elem for bf16 gradients (14 B for
     fp32 ones).  This library also writes the low half of its bf16-pair iterate
     (X0 = hi + lo, 2 B more), reported separately as the bytes it moves.
-    apply (when not fused): read W (4 B) and O = hi + lo (4 B), write W (4 B) = 12 B/elem.
-    Returns (momentum algorithmic, momentum moved, apply)."""
+    apply, the method's count: read W (4 B) and the bf16 O (2 B), write W (4 B) =
+    10 B/elem; the apply kernel reads O as the pair hi + lo (2 B more), reported
+    separately as the bytes it moves (12 B/elem).
+    Returns (momentum algorithmic, momentum moved, apply algorithmic, apply moved)."""
     g = 2 if w.grad_dtype == wl.BF16 else 4
-    return w.elements * (g + 4 + 4 + 2), w.elements * (g + 4 + 4 + 2 + 2), w.elements * 12
+    e = w.elements
+    return e * (g + 4 + 4 + 2), e * (g + 4 + 4 + 2 + 2), e * (4 + 2 + 4), e * (4 + 2 + 2 + 4)
 
 
 def update_gemm_flops(w: wl.Workload):
@@ -352,8 +355,9 @@ def measure(opt, groups, steps: int, warmup: int, world: int, dev, load_s: float
 
 
 def ns_figures(w: wl.Workload, ms_step: float, burst_ms: float, phases, steps: int, peaks, world: int = 1):
-    """Newton-Schulz throughput on both FLOP counts and the momentum kernel's HBM
-    throughput, each with the numbers it is computed from.
+    """Newton-Schulz throughput on both FLOP counts and the momentum and apply
+    kernels' HBM throughput (the method's byte counts, and the bytes the bf16-pair
+    iterate moves), each with the numbers it is computed from.
 
     nominal:   5 (4 m^2 n + 2 m^3) per matrix (the metric's count), over the step time;
     symmetric: 5 (3 m^2 n + m^3), the work left when the two symmetric products are
@@ -368,7 +372,9 @@ def ns_figures(w: wl.Workload, ms_step: float, burst_ms: float, phases, steps: i
     gemm_ms = sum(phases[k][0] for k in ("gram", "poly", "update")) / steps
     ns_ms = max(ms_step - mom_ms, 1e-9)
     ns_burst_ms = max(burst_ms - mom_ms, 1e-9)
-    b_mom, b_mom_moved, _ = elementwise_bytes(w)
+    b_mom, b_mom_moved, b_app, b_app_moved = elementwise_bytes(w)
+    apply_fused = phases["apply"][1] == 0
+    app_ms = phases["apply"][0] / max(phases["apply"][1], 1)
     sym = flops_sym / (ns_ms * 1e-3) / 1e12
     return {
         "ns5_tflops_nominal": round(flops_nom * world / (ms_step * 1e-3) / 1e12, 2),
@@ -386,6 +392,13 @@ def ns_figures(w: wl.Workload, ms_step: float, burst_ms: float, phases, steps: i
         "momentum_bytes_per_elem": b_mom / w.elements,
         "momentum_gbs_moved": round(b_mom_moved / (mom_ms * 1e-3) / 1e9, 1),
         "momentum_moved_bytes_per_elem": b_mom_moved / w.elements,
+        "apply": "fused into the epilogue of the last update GEMM" if apply_fused else "apply_kernel",
+        "apply_ms": None if apply_fused else round(app_ms, 4),
+        "apply_gbs": None if apply_fused else round(b_app / (app_ms * 1e-3) / 1e9, 1),
+        "apply_frac_of_hbm": None if apply_fused else round(b_app / (app_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
+        "apply_bytes_per_elem": b_app / w.elements,
+        "apply_gbs_moved": None if apply_fused else round(b_app_moved / (app_ms * 1e-3) / 1e9, 1),
+        "apply_moved_bytes_per_elem": b_app_moved / w.elements,
     }
 
 
@@ -445,9 +458,6 @@ def run_ours(args, w):
     flops_nom = w.ns_flops_nominal()
     value = flops_nom * world / (ms_step * 1e-3) / 1e12
     launches = sum(n for (_, n) in phases.values())
-    _, _, b_app = elementwise_bytes(w)
-    apply_fused = phases["apply"][1] == 0
-    app_ms = phases["apply"][0] / max(phases["apply"][1], 1)
     upd_ms = phases["update"][0] / max(phases["update"][1], 1)
     upd_tflops = update_gemm_flops(w) / (upd_ms * 1e-3) / 1e12
     # the timed region runs after >= 1 s of continuous load: the sustained bf16 peak
@@ -497,9 +507,6 @@ def run_ours(args, w):
     line.update(nsf)
     line.update({
         "momentum_peak": f"{peaks['hbm_gbs']} GB/s ({peak_src} HBM copy)",
-        "apply_gbs": None if apply_fused else round(b_app / (app_ms * 1e-3) / 1e9, 1),
-        "apply_frac_of_hbm": None if apply_fused else round(b_app / (app_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4),
-        "apply": "fused into the epilogue of the last update GEMM" if apply_fused else "apply_kernel",
         "phase_ms_per_step": {k: round(v[0] / args.steps, 4) for k, v in phases.items()},
         "roofline": {"kernel": "update GEMM X' = P X + aX (ns_gemm_tc2_kernel<2>)", "bound": "tensor",
                      "achieved": round(upd_tflops, 2), "peak": tpeak, "unit": "TFLOP/s",

@@ -27,11 +27,13 @@ def test_cpu_baseline_record():
 
 
 def test_elementwise_bytes_per_element():
-    """The method's count for the momentum kernel: G 2 (bf16) or 4 (fp32), B 4 + 4,
-    X0 2 = 12 (14) B/elem; the bf16-pair iterate moves 2 B/elem more."""
+    """The method's counts: momentum G 2 (bf16) or 4 (fp32), B 4 + 4, X0 2 = 12 (14)
+    B/elem; apply W 4 + 4, O 2 = 10 B/elem.  The bf16-pair iterate moves 2 B/elem more
+    in each (X0's lo written, O's lo read)."""
     w = wl.get("square4096")
-    mom, moved, app = bench.elementwise_bytes(w)
-    assert mom == 12 * w.elements and moved == 14 * w.elements and app == 12 * w.elements
+    mom, moved, app, app_moved = bench.elementwise_bytes(w)
+    assert mom == 12 * w.elements and moved == 14 * w.elements
+    assert app == 10 * w.elements and app_moved == 12 * w.elements
     t = wl.get("tiny")
     assert bench.elementwise_bytes(t)[0] == 14 * t.elements
 
@@ -42,7 +44,7 @@ def test_ns_figures_follow_their_stated_counts():
     peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0}
     steps = 4
     phases = {"momentum_norm": (0.2, 4), "norm_finalize": (0.0, 0), "gram": (1.2, 20), "poly": (1.2, 20),
-              "update": (2.0, 20), "apply": (0.0, 0)}
+              "update": (2.0, 20), "apply": (0.16, 4)}
     f = bench.ns_figures(w, 1.25, 1.10, phases, steps, peaks)
     m = 4096.0
     sym = 5 * (3 * m ** 3 + m ** 3)
@@ -53,6 +55,13 @@ def test_ns_figures_follow_their_stated_counts():
     assert abs(f["ns5_symmetric"]["tflops_burst"] - round(sym / 1.05e-3 / 1e12, 2)) < 1e-6
     assert abs(f["momentum_gbs"] - round(12 * w.elements / 0.05e-3 / 1e9, 1)) < 1e-6
     assert f["momentum_bytes_per_elem"] == 12 and f["momentum_moved_bytes_per_elem"] == 14
+    assert f["apply"] == "apply_kernel" and abs(f["apply_ms"] - 0.04) < 1e-12
+    assert abs(f["apply_gbs"] - round(10 * w.elements / 0.04e-3 / 1e9, 1)) < 1e-6
+    assert abs(f["apply_frac_of_hbm"] - round(10 * w.elements / 0.04e-3 / 1e9 / 6000.0, 4)) < 1e-9
+    assert abs(f["apply_gbs_moved"] - round(12 * w.elements / 0.04e-3 / 1e9, 1)) < 1e-6
+    fused = dict(phases, apply=(0.0, 0))
+    g = bench.ns_figures(w, 1.25, 1.10, fused, steps, peaks)
+    assert g["apply_gbs"] is None and g["apply"].startswith("fused")
     nominal = 5 * (4 * m ** 3 + 2 * m ** 3)
     assert abs(f["ns5_tflops_nominal"] - round(nominal / 1.25e-3 / 1e12, 2)) < 1e-6
     assert abs(f["ns5_tflops_phase_sum"] - round(nominal / 1.1e-3 / 1e12, 2)) < 1e-6
