@@ -63,6 +63,7 @@ struct Plan {
     int4* d_units[3] = {nullptr, nullptr, nullptr};
     int* d_unit_begin[3] = {nullptr, nullptr, nullptr};
     int unit_clusters = 0;
+    int active[3] = {0, 0, 0};           // per phase: clusters that have units (launched)
     float* d_sk_partial = nullptr;
     int* d_sk_count = nullptr;
     int* d_sk_flag = nullptr;
@@ -366,8 +367,21 @@ bool is_bf16_path(const muon_handle* h) { return h->cfg.precision == MUON_PREC_B
 
 // Persistent grid: one CTA (or one two-CTA cluster) per tile, at most one per SM.
 // The two-CTA kernel runs one pair per unit list (lists are built for max_clusters).
-int gemm_grid(const muon_handle* h, int ntiles) {
-    if (h->pair) return 2 * h->max_clusters;
+// Clusters of a unit plan that have work.  build_units deals from cluster 0, so they
+// are a prefix; a phase with fewer units than clusters then launches only those and
+// the idle clusters skip their set-up (TMEM allocation, barriers, cluster sync).  A
+// plan whose busy clusters are not a prefix launches every cluster.
+int active_clusters(const UnitPlan& up, int clusters) {
+    int k = 0;
+    while (k < clusters && up.begin[k + 1] > up.begin[k]) ++k;
+    for (int c = k; c < clusters; ++c)
+        if (up.begin[c + 1] > up.begin[c]) return clusters;
+    return k;
+}
+
+// pair: two CTAs per cluster that has units (`active`, 0 = all clusters)
+int gemm_grid(const muon_handle* h, int ntiles, int active = 0) {
+    if (h->pair) return 2 * (active > 0 ? active : h->max_clusters);
     return std::min(ntiles, h->num_sms);
 }
 
@@ -445,6 +459,7 @@ muon_status ensure_plan(muon_handle* h, const std::vector<int>& shapes, cudaStre
                 }
                 upl[ph] = build_units(*lists[ph], kb, h->max_clusters, tc_gemm_split_tiles() != 0, true);
                 sk_slots = std::max(sk_slots, upl[ph].nslots);
+                P.active[ph] = active_clusters(upl[ph], h->max_clusters);
             }
             P.unit_clusters = h->max_clusters;
         }
@@ -660,10 +675,10 @@ muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStrea
             gp.tiles = P.d_tiles_gram; gp.ntiles = P.n_gram; gp.alpha = 1.f; gp.beta = 0.f;
             gp.units = P.d_units[0]; gp.unit_begin = P.d_unit_begin[0]; gp.epoch = ++h->epoch;
             gp.scale = it == 0 ? P.d_scale : nullptr;
-            TIMED(h, 2, s, launch_tc_gemm(MODE_GRAM, h->pair, gp, gemm_grid(h, P.n_gram), s, P.var[0]));
+            TIMED(h, 2, s, launch_tc_gemm(MODE_GRAM, h->pair, gp, gemm_grid(h, P.n_gram, P.active[0]), s, P.var[0]));
             gp.tiles = P.d_tiles_poly; gp.ntiles = P.n_poly; gp.alpha = c.ns_c; gp.beta = c.ns_b; gp.scale = nullptr;
             gp.units = P.d_units[1]; gp.unit_begin = P.d_unit_begin[1]; gp.epoch = ++h->epoch;
-            TIMED(h, 3, s, launch_tc_gemm(MODE_POLY, h->pair, gp, gemm_grid(h, P.n_poly), s, P.var[1]));
+            TIMED(h, 3, s, launch_tc_gemm(MODE_POLY, h->pair, gp, gemm_grid(h, P.n_poly, P.active[1]), s, P.var[1]));
             gp.tiles = P.d_tiles_upd; gp.ntiles = P.n_upd; gp.alpha = 1.f; gp.beta = c.ns_a;
             gp.units = P.d_units[2]; gp.unit_begin = P.d_unit_begin[2]; gp.epoch = ++h->epoch;
             gp.scale = it == 0 ? P.d_scale : nullptr;
@@ -674,7 +689,7 @@ muon_status run_pipeline(muon_handle* h, bool momentum, bool copy_out, cudaStrea
                 gp.lr = c.lr;
                 gp.segs = P.d_segs;
             }
-            TIMED(h, 4, s, launch_tc_gemm(MODE_UPDATE, h->pair, gp, gemm_grid(h, P.n_upd), s, P.var[2]));
+            TIMED(h, 4, s, launch_tc_gemm(MODE_UPDATE, h->pair, gp, gemm_grid(h, P.n_upd, P.active[2]), s, P.var[2]));
         } else {
             for (size_t g = 0; g < P.dims.size(); ++g) {
                 const GroupDims& d = P.dims[g];
@@ -1235,8 +1250,8 @@ muon_status muon_ns_phase_run(muon_handle* h, const muon_ns_phase_args* a, void*
     gp.scale = nullptr;
     gp.err = h->d_err;
     const int mode = phase == MUON_NS_GRAM ? MODE_GRAM : phase == MUON_NS_POLY ? MODE_POLY : MODE_UPDATE;
-    CUDA_TRY(h, launch_tc_gemm(mode, h->pair, gp, gemm_grid(h, gp.ntiles), s,
-                               tc_gemm_var(mode, phase == MUON_NS_GRAM ? n : m)));
+    CUDA_TRY(h, launch_tc_gemm(mode, h->pair, gp, gemm_grid(h, gp.ntiles, h->pair ? active_clusters(up, h->max_clusters) : 0),
+                               s, tc_gemm_var(mode, phase == MUON_NS_GRAM ? n : m)));
     return MUON_OK;
 }
 
