@@ -38,6 +38,53 @@ def _step_one(shapes, cfg, grads, weights, dtype=torch.float32):
     return out
 
 
+@pytest.mark.parametrize("precision", [mb.PREC_BF16, mb.PREC_FP32_DEBUG])
+def test_rank_deficient_gradients(precision):
+    """The method's degenerate inputs: Newton-Schulz maps zero singular values to
+    zero, so a rank-r gradient (here rank 1, 5 and 64) gives a rank-r direction, and
+    zero rows of G give zero rows of O.
+
+    In finite precision the iteration amplifies whatever rounding leaves in the null
+    space: p(s) ~ a s for small s, so a component entering at iteration j grows by
+    a^(5-j+1) and the sum over the five iterations is at most sum_j a^j ~ 580
+    (a = 3.4445).  fp32 GEMMs at K <= 1024 leave ~ sqrt(K) 2^-24 ~ 2e-6 of ||X|| per
+    iteration, hence a null-space part up to ~1.2e-3 of ||O|| in the fp32 debug path
+    (2e-3 below); the bf16-pair iterate (~2^-17 per element) gives ~1e-2, under the
+    bf16 tolerance.  So: the part of O in G's column space matches the oracle within
+    the path's tolerance, the rest stays under that bound, and the zero rows are zero
+    exactly (every product that forms them is a product with zero)."""
+    rng = np.random.default_rng(21)
+    cases = [((512, 256), 1), ((256, 768), 5), ((1024, 384), 64), ((300, 300), None)]
+    shapes = [sh for sh, _ in cases]
+    G = []
+    for (r, c), k in cases:
+        if k is None:
+            g = rng.standard_normal((r, c)).astype(np.float32)
+            g[::7][:40] = 0.0                                  # 40 zero rows, spread out
+        else:
+            g = (rng.standard_normal((r, k)) @ rng.standard_normal((k, c))).astype(np.float32)
+        G.append(g)
+    W0 = [0.02 * rng.standard_normal(sh) for sh in shapes]
+    W, B, O = _step_one(shapes, mb.config(precision=precision), G, W0)
+    tol = TOL_O[precision]
+    null_tol = tol if precision == mb.PREC_BF16 else 2e-3
+    for i, ((r, c), k) in enumerate(cases):
+        res = oracle.muon_step(W0[i].astype(np.float32).astype(np.float64), G[i].astype(np.float64),
+                               np.zeros((r, c)), lr=0.02, momentum=0.95, nesterov=True, eps=1e-7)
+        assert np.array_equal(B[i], G[i].astype(np.float64))        # first step from B = 0: B = G exactly
+        if k is None:
+            zero = np.all(G[i] == 0.0, axis=1)
+            assert zero.sum() == 40
+            assert np.all(O[i][zero] == 0.0)
+            assert rel_fro(O[i], res["O"]) <= tol, (r, c, rel_fro(O[i], res["O"]))
+            continue
+        Ur = np.linalg.svd(G[i].astype(np.float64), full_matrices=False)[0][:, :k]
+        inside = Ur @ (Ur.T @ O[i])
+        assert rel_fro(inside, Ur @ (Ur.T @ res["O"])) <= tol, (r, c, k, rel_fro(inside, Ur @ (Ur.T @ res["O"])))
+        null = np.linalg.norm(O[i] - inside) / np.linalg.norm(O[i])
+        assert null <= null_tol, (r, c, k, null)
+
+
 ODD = [(37, 1000), (1000, 37), (1, 64), (64, 1), (1, 1), (129, 257), (300, 129), (8, 8),
        (1001, 72), (130, 8)]          # tall with 8-aligned columns: vector transpose, ragged rows
 
