@@ -85,6 +85,36 @@ def test_rank_deficient_gradients(precision):
         assert null <= null_tol, (r, c, k, null)
 
 
+CUBIC = (1.5, -0.5, 0.0)      # the classical cubic Newton-Schulz step X <- 1.5X - 0.5XX^TX
+
+
+@pytest.mark.parametrize("ns_steps,coeffs,precision", [
+    (1, None, mb.PREC_BF16), (2, None, mb.PREC_BF16), (3, None, mb.PREC_BF16), (4, None, mb.PREC_BF16),
+    (6, None, mb.PREC_BF16), (2, None, mb.PREC_FP32_DEBUG), (4, CUBIC, mb.PREC_BF16), (3, CUBIC, mb.PREC_FP32_DEBUG)])
+def test_iteration_count_and_coefficients(ns_steps, coeffs, precision):
+    """Other iteration counts (odd and even: the final iterate sits in either buffer of
+    the ping-pong pair) and other coefficients (the cubic step, c = 0) against the
+    oracle run with the same settings, on a wide, a tall (transposed) and a ragged
+    matrix in one grouped call; W from the GPU's O by the oracle's update formula."""
+    rng = np.random.default_rng(31 + ns_steps)
+    shapes = [(256, 512), (640, 384), (520, 264)]
+    G = [rng.standard_normal(sh).astype(np.float32) for sh in shapes]
+    W0 = [0.02 * rng.standard_normal(sh) for sh in shapes]
+    kw = dict(ns_steps=ns_steps, precision=precision, weight_decay=0.1)
+    if coeffs is not None:
+        kw.update(ns_a=coeffs[0], ns_b=coeffs[1], ns_c=coeffs[2])
+    W, B, O = _step_one(shapes, mb.config(**kw), G, W0)
+    for i, sh in enumerate(shapes):
+        w0 = W0[i].astype(np.float32).astype(np.float64)
+        res = oracle.muon_step(w0, G[i].astype(np.float64), np.zeros(sh), lr=0.02, momentum=0.95, nesterov=True,
+                               weight_decay=0.1, ns_steps=ns_steps, eps=1e-7,
+                               coeffs=coeffs if coeffs is not None else oracle.NS_COEFFS)
+        assert rel_fro(O[i], res["O"]) <= TOL_O[precision], (sh, rel_fro(O[i], res["O"]))
+        assert np.array_equal(B[i], G[i].astype(np.float64))
+        Wexp = oracle.apply_update(w0, O[i], 0.02, 0.1, 1.0)
+        assert np.max(np.abs(W[i] - Wexp) / (np.abs(w0) + 0.02 * np.abs(O[i]) + 1e-30)) <= 1e-6
+
+
 ODD = [(37, 1000), (1000, 37), (1, 64), (64, 1), (1, 1), (129, 257), (300, 129), (8, 8),
        (1001, 72), (130, 8)]          # tall with 8-aligned columns: vector transpose, ragged rows
 
