@@ -26,7 +26,7 @@
 //  ns_gemm_tc2_kernel (a cluster of two CTAs per 256 x 256 tile), 384 threads per CTA:
 //   warp 0      TMA producer: each CTA stages its 128 rows of A and its 128 columns of B
 //               (a ring of 4 or 5 stages of 16 + 16 KiB); the odd CTA's loads complete
-//               on the even CTA's barrier; no multicast form is used.
+//               on the even CTA's barrier; each load fills one CTA's shared memory.
 //   warp 1      the even CTA's elected thread issues tcgen05.mma.cta_group::2 (M=256,
 //               N=256, K=16), which reads both CTAs' shared memory; each CTA's TMEM
 //               receives its 128 accumulator rows; completion is committed to the

@@ -1,4 +1,4 @@
-// ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarrier, TMA (no multicast),
+// ptx.cuh -- thin inline-PTX wrappers for sm_100a: mbarrier, TMA (each load fills one CTA),
 // tcgen05 (TMEM alloc, MMA, commit, loads) and a bounded barrier wait.
 //
 // Every wait on an mbarrier is bounded: after MUON_WAIT_NS nanoseconds of
@@ -90,7 +90,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     }
 }
 
-// ---------------------------------------------------------------- TMA (plain tiled loads, no multicast)
+// ---------------------------------------------------------------- TMA (plain tiled loads into one CTA)
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
     asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
@@ -109,11 +109,10 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, ui
         : "memory");
 }
 
-// 3-D tiled store from this CTA's shared memory (no multicast form exists for
-// stores).  Elements of the box outside the tensor are not written.  Completion is
-// tracked per issuing thread with bulk groups (bulk_commit / bulk_wait_*).  Every
-// store in this library starts at non-negative coordinates, c0 a multiple of 32
-// bf16 elements (64 bytes).
+// 3-D tiled store from this CTA's shared memory.  Elements of the box outside the
+// tensor are not written.  Completion is tracked per issuing thread with bulk
+// groups (bulk_commit / bulk_wait_*).  Every store in this library starts at
+// non-negative coordinates, c0 a multiple of 32 bf16 elements (64 bytes).
 __device__ __forceinline__ void tma_store_3d(const void* tmap, const void* smem_src, int c0, int c1, int c2) {
     asm volatile(
         "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
@@ -236,8 +235,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(uint32_t M, uint32_t N, ui
 // A cluster of two CTAs shares one 256-row MMA: each CTA stages its half of A and
 // of B in its own shared memory, the even CTA (rank 0) issues the MMA, and each
 // CTA's TMEM receives its 128 accumulator rows.  Barriers of the other CTA are
-// addressed through shared::cluster addresses obtained with mapa; no load or
-// arrive in this file uses a multicast form.
+// addressed through shared::cluster addresses obtained with mapa; every load
+// and arrive in this file targets a single CTA.
 namespace muon {
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
