@@ -79,3 +79,14 @@ def test_fused_copy_out_matches_standalone_and_oracle(dtype, monkeypatch):
             assert torch.equal(Of, Os)
             ref = oracle.newton_schulz(M.float().cpu().numpy().astype(np.float64), eps=1e-7)
             assert rel_fro(Of.cpu().numpy().astype(np.float64), ref) <= TOL_O[mb.PREC_BF16]
+
+
+@pytest.mark.parametrize("fused", [False, True])
+def test_one_cta_kernel_whole_step_parity(fused, monkeypatch):
+    """The selectable one-CTA GEMM kernel (MUON_GEMM_PAIR=0) through a whole step:
+    GPT-2-small (all 72 matrices) against the oracle, with the apply kernel and with
+    its own fused weight update."""
+    monkeypatch.setenv("MUON_GEMM_PAIR", "0")
+    monkeypatch.setenv("MUON_FUSED_APPLY", "1" if fused else "0")
+    StepParity(wl.get(2), mb.PREC_BF16, steps=1).run().assert_ok()
+
