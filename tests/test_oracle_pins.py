@@ -88,6 +88,23 @@ def test_newton_schulz_rank_deficient_closed_form():
     assert np.all(s[5:] < 1e-10 * s[0])          # zero singular values stay zero (p(0) = 0)
 
 
+@pytest.mark.parametrize("steps,coeffs", [(1, oracle.NS_COEFFS), (3, oracle.NS_COEFFS), (6, oracle.NS_COEFFS),
+                                          (4, (1.5, -0.5, 0.0)), (2, (2.0, -1.5, 0.5))])
+def test_other_steps_and_coefficients_follow_the_closed_form(steps, coeffs):
+    """The iteration count and (a, b, c) are parameters of one polynomial map,
+    U p^steps(S / ||M||_F) V^T with p(s) = a s + b s^3 + c s^5: for the quintic of
+    section 4 at other counts and for other coefficients (the classical cubic step
+    (1.5, -0.5, 0)).  muon_step passes both on: its first step from B = 0 orthogonalises
+    the Nesterov direction U = G + mu G."""
+    rng = np.random.default_rng(steps)
+    M = rng.standard_normal((24, 40))
+    assert rel(oracle.newton_schulz(M, steps=steps, coeffs=coeffs, eps=0.0), closed_form_ns(M, steps, 0.0, coeffs)) < 1e-10
+    G = rng.standard_normal((40, 24))
+    res = oracle.muon_step(np.zeros((40, 24)), G, np.zeros((40, 24)), lr=0.02, momentum=0.9, nesterov=True,
+                           ns_steps=steps, coeffs=coeffs, eps=0.0)
+    assert rel(res["O"], closed_form_ns(G + 0.9 * G, steps, 0.0, coeffs)) < 1e-10
+
+
 def test_newton_schulz_eps_enters_as_norm_plus_eps():
     M = np.random.default_rng(5).standard_normal((6, 10)) * 1e-6
     eps = 1e-7
