@@ -367,18 +367,6 @@ bool is_bf16_path(const muon_handle* h) { return h->cfg.precision == MUON_PREC_B
 
 // Persistent grid: one CTA (or one two-CTA cluster) per tile, at most one per SM.
 // The two-CTA kernel runs one pair per unit list (lists are built for max_clusters).
-// Clusters of a unit plan that have work.  build_units deals from cluster 0, so they
-// are a prefix; a phase with fewer units than clusters then launches only those and
-// the idle clusters skip their set-up (TMEM allocation, barriers, cluster sync).  A
-// plan whose busy clusters are not a prefix launches every cluster.
-int active_clusters(const UnitPlan& up, int clusters) {
-    int k = 0;
-    while (k < clusters && up.begin[k + 1] > up.begin[k]) ++k;
-    for (int c = k; c < clusters; ++c)
-        if (up.begin[c + 1] > up.begin[c]) return clusters;
-    return k;
-}
-
 // pair: two CTAs per cluster that has units (`active`, 0 = all clusters)
 int gemm_grid(const muon_handle* h, int ntiles, int active = 0) {
     if (h->pair) return 2 * (active > 0 ? active : h->max_clusters);

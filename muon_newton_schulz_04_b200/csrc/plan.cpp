@@ -123,6 +123,15 @@ UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kbl
     return up;
 }
 
+int active_clusters(const UnitPlan& up, int clusters) {
+    if ((int)up.begin.size() < clusters + 1) return clusters;
+    int k = 0;
+    while (k < clusters && up.begin[k + 1] > up.begin[k]) ++k;
+    for (int c = k; c < clusters; ++c)
+        if (up.begin[c + 1] > up.begin[c]) return clusters;
+    return k;
+}
+
 std::string check_plan(const std::vector<GroupDims>& groups, int phase, int bm, int bn, int bk,
                        const std::vector<Tile>& tiles, const std::vector<int>& kblocks, const UnitPlan* up,
                        int clusters) {

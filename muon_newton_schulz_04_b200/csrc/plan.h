@@ -56,6 +56,13 @@ struct UnitPlan {
 UnitPlan build_units(const std::vector<Tile>& tiles, const std::vector<int>& kblocks, int clusters, bool split,
                      bool half_tail = false);
 
+// Clusters of a unit plan that have work.  build_units deals from cluster 0, so they
+// are a prefix; a phase with fewer units than clusters then launches only those and
+// the idle clusters skip their set-up (TMEM allocation, barriers, cluster sync).
+// Returns `clusters` when the busy clusters are not a prefix (every cluster is
+// launched), 0 when no cluster has work.
+int active_clusters(const UnitPlan& up, int clusters);
+
 // Host-side check of a plan before anything is launched with it: the tile list of
 // `phase` holds every tile it should exactly once (in range, and for GRAM / POLY
 // touching col >= row), kblocks[i] is tile i's K-block count, and -- when `up` is

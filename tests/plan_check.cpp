@@ -105,6 +105,23 @@ int main() {
             if (u.n_half == 2) { u.n_half = 1; break; }
         expect(!check(h, 2, 3).empty(), "halves that do not pair up");
     }
+    // clusters launched: the busy ones form a prefix of the deal
+    {
+        Case few = make({{256, 512, 1}}, 2, 74, false);           // 2 update tiles on 74 clusters
+        expect(active_clusters(few.up, 74) == 2, "two tiles keep two clusters busy");
+        Case full = make({{4096, 4096, 1}}, 2, 74, false);        // 256 tiles: every cluster
+        expect(active_clusters(full.up, 74) == 74, "a full plan keeps every cluster");
+        Case half = make({{1024, 256, 1}}, 2, 3, false);           // 3 whole tiles + 2 halves on 3 clusters
+        expect(active_clusters(half.up, 3) == 3, "halves keep their clusters");
+        Case gap = few;                                            // work moved behind an idle cluster
+        gap.up.begin = std::vector<int>(75, 2);
+        gap.up.begin[0] = 0; gap.up.begin[1] = 1; gap.up.begin[2] = 1;
+        for (int c = 3; c <= 74; ++c) gap.up.begin[c] = 2;
+        expect(active_clusters(gap.up, 74) == 74, "busy clusters that are not a prefix launch all");
+        UnitPlan none;
+        none.begin = std::vector<int>(75, 0);
+        expect(active_clusters(none, 74) == 0, "no work, no cluster");
+    }
     std::printf(failures == 0 ? "plan check ok\n" : "plan check: %d failures\n", failures);
     return failures == 0 ? 0 : 1;
 }
