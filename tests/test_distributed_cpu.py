@@ -61,11 +61,12 @@ def _spawn(tmp_path, world, steps, variant):
 
 
 @pytest.mark.timeout(300)
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 8])
 def test_sharded_step_gloo(tmp_path, world):
     """Whole-matrix ownership with the bf16 direction payload: every rank ends with
     the weights of a one-process run that applies the same bf16 directions.  World 3
-    gives shards of unequal element counts (the packed buffer is padded)."""
+    gives shards of unequal element counts (the packed buffer is padded); world 8 one
+    matrix per rank."""
     steps = 2
     outs = _spawn(tmp_path, world, steps, "sharded")
     ref = dist_worker.reference(steps, payload_dtype=torch.bfloat16)
@@ -77,12 +78,13 @@ def test_sharded_step_gloo(tmp_path, world):
 
 
 @pytest.mark.timeout(300)
-@pytest.mark.parametrize("world", [2, 3])
+@pytest.mark.parametrize("world", [2, 3, 8])
 def test_zero1_step_gloo(tmp_path, world):
     """Row-sliced momentum (ZeRO-1 Distributed Muon): gather the direction rows,
     orthogonalise full matrices, update own rows, gather W.  Every rank ends with
     the weights of the one-process oracle step, bitwise, and its momentum rows are
-    that run's momentum rows.  World 3 splits 8-row and 5-row matrices unevenly."""
+    that run's momentum rows.  World 3 splits 8-row and 5-row matrices unevenly;
+    world 8 leaves three ranks with no rows of the 5-row matrix."""
     steps = 2
     outs = _spawn(tmp_path, world, steps, "zero1")
     W_ref = dist_worker.initial_weights()
